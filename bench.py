@@ -1,0 +1,312 @@
+"""Benchmark: last-scale block-sparse cross-scale attention on B200.
+
+One step = the whole hot path for the Infinity-2B-like last scale (64x64
+queries over the 10521-key prefix, B2 H16 D128, 128x128 blocks): the CSLA
+block-list build followed by the block-sparse attention forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  ``value`` is kept-block TFLOP/s of the whole job
+(4 * n_q * n_k * D per kept block, valid elements only, summed over all ranks)
+divided by the slowest rank's device time.  Multi-GPU runs (torchrun) give
+every rank its own independent batch of the same size (weak scaling, no
+collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_cross_sparvar_b200 import inputs  # noqa: E402
+
+WORKLOAD = dict(name="infinity2b_last_scale_64x64", sides=inputs.INFINITY_SIDES, q_scale=12,
+                B=2, H=16, D=128, n_sink_scales=5, radius_prev=2, radius_own=4, block=128)
+FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    hbm=p["hbm_gbs"], source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def kept_flops_from_lists(cnt, idx, nq, L, bq, bk, D):
+    total = 0
+    for qb in range(cnt.shape[0]):
+        nqr = min((qb + 1) * bq, nq) - qb * bq
+        for kb in idx[qb, :cnt[qb]]:
+            nkr = min((int(kb) + 1) * bk, L) - int(kb) * bk
+            total += 4 * nqr * nkr * D
+    return total
+
+
+def start_clock_sampler(path):
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    try:
+        f = open(path, "w")
+        return subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                 "-lms", "100"], stdout=f, stderr=subprocess.DEVNULL), f
+    except Exception:
+        return None, None
+
+
+def stop_clock_sampler(proc, f, path, gpu_index):
+    if proc is None:
+        return None
+    proc.terminate()
+    try:
+        proc.wait(timeout=5)
+    except Exception:
+        proc.kill()
+    f.close()
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in open(path):
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9 or parts[0] != str(gpu_index):
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = max(mx, float(parts[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "samples": len(sm),
+            "reasons": sorted(reasons)}
+
+
+def cpu_baseline(wl, budget_s=12.0, seed=0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload:
+    one (batch, head) and as many query blocks as fit in ``budget_s``."""
+    from oracle import sparvar_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    sides, k = wl["sides"], wl["q_scale"]
+    d = inputs.make_qkv(seed, 1, 1, sides, wl["D"], wl["n_sink_scales"])
+    off = d["offsets"]
+    f64 = lambda a: a.astype(np.float64)  # noqa: E731
+    q = f64(d["qf"][0, 0, off[k]:off[k + 1]])
+    kk = f64(d["kf"][0, 0, :off[k + 1]])
+    vv = f64(d["vf"][0, 0, :off[k + 1]])
+    bq = wl["block"]
+    t0 = time.perf_counter()
+    cnt, idx, blk = orc.build_csla_mask(sides, k, wl["n_sink_scales"], wl["radius_prev"],
+                                        wl["radius_own"], bq, bq)
+    nq, L = q.shape[0], kk.shape[0]
+    flops, done = 0, 0
+    while done < blk.shape[0] and time.perf_counter() - t0 < budget_s:
+        rows = np.arange(done * bq, min((done + 1) * bq, nq))
+        orc.masked_attention_rows(rows, q, kk, vv, blk, bq, bq)
+        sub = np.zeros_like(blk)
+        sub[done] = blk[done]
+        flops += orc.kept_flops(sub, nq, L, bq, bq, wl["D"])
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"1 of {wl['B'] * wl['H']} (batch, head) pairs, {done} of {blk.shape[0]} query "
+                      f"blocks, CSLA mask build included; numpy fp64 ({dt:.1f} s)",
+            "seconds": dt}
+
+
+def run_reference(args, wl, rank, world):
+    if world > 1 and rank != 0:
+        return
+    per_step = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        res = cpu_baseline(wl, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)), seed=0)
+        if i >= args.warmup:
+            per_step.append(res)
+    val = float(np.mean([r["value"] for r in per_step]))
+    line = {"impl": "reference", "metric": "last-scale block-sparse attn ms and kept-block TFLOP/s "
+            "(% of bf16 TC peak)", "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": float(np.mean([r["seconds"] for r in per_step]) * 1e3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl["name"], "B": wl["B"], "H": wl["H"],
+                                            "Lq": 4096, "Lkv": 10521, "D": wl["D"],
+                                            "block": wl["block"], "mask": "csla"},
+            "cpu_baseline": {k: per_step[-1][k] for k in ("kind", "cores", "sample")} | {"value": val,
+                                                                                      "unit": "TFLOP/s"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOAD
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from block_sparse_cross_sparvar_b200 import ops
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    sides, k, D, B, H, bq = wl["sides"], wl["q_scale"], wl["D"], wl["B"], wl["H"], wl["block"]
+    d = inputs.make_qkv(rank, B, H, sides, D, wl["n_sink_scales"])
+    off = d["offsets"]
+    nq, L = off[k + 1] - off[k], off[k + 1]
+    to_host = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    hq = to_host(d["q"][:, :, off[k]:off[k + 1]]).pin_memory()
+    hk = to_host(d["k"]).pin_memory()
+    hv = to_host(d["v"]).pin_memory()
+    del d
+    q, kk, vv = hq.to(dev), hk.to(dev), hv.to(dev)
+    o = torch.empty_like(q)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(qq, kk_, vv_, out):
+        cnt, idx, _ = ops.sparvar_build_csla_mask(sides, k, wl["n_sink_scales"], wl["radius_prev"],
+                                                  wl["radius_own"], bq, bq, device=dev)
+        ops.sparvar_block_sparse_attn_fwd(qq, kk_, vv_, cnt, idx, bq, bq, out=out, dev_status=status)
+        return cnt, idx
+
+    cnt, idx = step(q, kk, vv, o)
+    torch.cuda.synchronize()
+    cnt_h, idx_h = cnt.cpu().numpy(), idx.cpu().numpy()
+    flops_step = kept_flops_from_lists(cnt_h, idx_h, nq, L, bq, bq, D) * B * H
+    dense_flops = 4 * nq * L * D * B * H
+    nqb, nkb = idx_h.shape
+
+    for _ in range(args.warmup):
+        step(q, kk, vv, o)
+    torch.cuda.synchronize()
+
+    clocks_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/sparvar_clocks_{rank}.csv"
+    sampler, sf = start_clock_sampler(clocks_path) if rank == 0 else (None, None)
+    time.sleep(0.3 if sampler else 0)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i)  # evict inputs from the 126 MB L2 between steps (not timed)
+        e0, e1, e2 = ev[i]
+        e0.record()
+        cnt_i, idx_i, _ = ops.sparvar_build_csla_mask(sides, k, wl["n_sink_scales"],
+                                                      wl["radius_prev"], wl["radius_own"], bq, bq,
+                                                      device=dev)
+        e1.record()
+        ops.sparvar_block_sparse_attn_fwd(q, kk, vv, cnt_i, idx_i, bq, bq, out=o, dev_status=status)
+        e2.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    attn_ms = [b_.elapsed_time(c) for _, b_, c in ev]
+    mask_ms = [a.elapsed_time(b_) for a, b_, _ in ev]
+    clocks = stop_clock_sampler(sampler, sf, clocks_path, torch.cuda.current_device()) if rank == 0 else None
+
+    # end to end through the public API: pinned host inputs -> device -> result -> host
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    e2e_ms = []
+    for i in range(max(3, min(args.steps, 10))):
+        flush.fill_(i)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        q.copy_(hq, non_blocking=True)
+        kk.copy_(hk, non_blocking=True)
+        vv.copy_(hv, non_blocking=True)
+        step(q, kk, vv, o)
+        ho.copy_(o, non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize()
+        e2e_ms.append(s0.elapsed_time(s1))
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} after the bench")
+
+    t_step = float(np.mean(step_ms))
+    t_attn = float(np.mean(attn_ms))
+    t_e2e = float(np.mean(e2e_ms))
+    if world > 1:
+        tt = torch.tensor([t_step, t_attn, t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, t_attn, t_e2e = tt.tolist()
+    total_flops = flops_step * world
+    pk = peaks()
+    if rank == 0:
+        achieved = flops_step / (t_attn * 1e-3) / 1e12
+        line = {
+            "metric": "last-scale block-sparse attn ms and kept-block TFLOP/s (% of bf16 TC peak)",
+            "value": total_flops / (t_step * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step,
+            "attn_ms": t_attn, "mask_build_ms": float(np.mean(mask_ms)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl["name"], "B": B, "H": H, "Lq": nq, "Lkv": L, "D": D,
+                       "block_q": bq, "block_kv": bq, "mask": "csla sink<=5 r_prev=2 r_own=4",
+                       "kept_blocks": int(cnt_h.sum()), "total_blocks": int(nqb * nkb),
+                       "kept_flop_fraction": flops_step / dense_flops,
+                       "kept_gflop_per_step_per_gpu": flops_step / 1e9,
+                       "l2": "256 MB flush write between timed steps",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "block_sparse_attn_kernel<128,0>",
+                         "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16"],
+                         "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']}",
+                         "traffic": None},
+            "e2e": {"value": total_flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": t_e2e,
+                    "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+                    "d2h_bytes_per_step": int(ho.numel() * 2)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = {kk_: v for kk_, v in cpu_baseline(wl).items() if kk_ != "seconds"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+// Integer kernels that build and check KV-block lists:
+//   csla_mask_kernel      CSLA sink + cross-scale locality mask, one CTA per query block
+//   map_indices_kernel    CS4A proportional index mapping, one CTA per (b, h, dst query block)
+//   validate_lists_kernel range / order check of block lists, one warp per list
+// All three build a KV-block bitset in shared memory with atomicOr and then
+// compact it into an ascending list (-1 padded) with warp ballots.  Integer
+// only, so results are exact.
+#pragma once
+
+#include <cstdint>
+
+namespace sparvar {
+
+constexpr int kMaskThreads = 256;
+
+struct ScaleGeometry {
+  int n_scales;
+  int side[32];
+  int off[33];
+};
+
+// Set bits [k0, k1] (inclusive) of a shared bitset.
+__device__ __forceinline__ void set_bit_range(uint32_t* bits, int k0, int k1) {
+  if (k1 < k0) return;
+  for (int w = k0 >> 5; w <= (k1 >> 5); ++w) {
+    const int lo = max(k0 - w * 32, 0);
+    const int hi = min(k1 - w * 32, 31);
+    const uint32_t upto = hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u);
+    const uint32_t from = ~((1u << lo) - 1u);
+    atomicOr(&bits[w], upto & from);
+  }
+}
+
+// Compact a bitset of nkb bits into an ascending index row (warp 0 only).
+__device__ __forceinline__ void compact_bitset(const uint32_t* bits, int nkb, int32_t* idx_row,
+                                               int32_t* cnt_out, uint8_t* mask_row) {
+  const int lane = threadIdx.x & 31;
+  const int nwords = (nkb + 31) >> 5;
+  int base = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t word = w < nwords ? bits[w] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = base + incl - c;
+    uint32_t rest = word;
+    while (rest) {
+      const int bit = __ffs(rest) - 1;
+      rest &= rest - 1;
+      idx_row[pos++] = w * 32 + bit;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int i = base + lane; i < nkb; i += 32) idx_row[i] = -1;
+  if (mask_row) {
+    for (int i = lane; i < nkb; i += 32) mask_row[i] = (bits[i >> 5] >> (i & 31)) & 1u;
+  }
+  if (lane == 0) *cnt_out = base;
+}
+
+// ---------------------------------------------------------------- CSLA
+// For the query block's rows, each (query row i, scale m) pair contributes the
+// keys of scale m in rows [ci - r, ci + r] and columns [cl - r, ch + r], where
+// ci = floor(i*s_m/s_k) and [cl, ch] is the projection of the block's columns in
+// row i (the projection of consecutive columns moves by 0 or 1, so the union of
+// the per-query windows is that rectangle).  Each key row of the rectangle is a
+// contiguous token range, which sets a contiguous range of KV-block bits.
+__global__ void __launch_bounds__(kMaskThreads)
+    csla_mask_kernel(const ScaleGeometry g, int q_scale, int n_sink, int r_prev, int r_own,
+                     int block_q, int block_kv, int nkb, int32_t* kv_cnt, int32_t* kv_idx,
+                     uint8_t* blk_mask) {
+  extern __shared__ uint32_t bits[];
+  const int qb = blockIdx.x;
+  const int nwords = (nkb + 31) >> 5;
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bits[w] = 0u;
+  __syncthreads();
+
+  const int sk = g.side[q_scale];
+  const int nq = sk * sk;
+  const int q0 = qb * block_q;
+  const int q1 = min(q0 + block_q, nq) - 1;
+  const int i0 = q0 / sk, i1 = q1 / sk;
+  const int sink_scales = min(n_sink, q_scale + 1);
+  const int n_sink_tok = g.off[sink_scales];
+  if (threadIdx.x == 0 && n_sink_tok > 0) set_bit_range(bits, 0, (n_sink_tok - 1) / block_kv);
+
+  const int m_first = n_sink;
+  const int num_m = q_scale - m_first + 1;
+  if (num_m > 0) {
+    const int num_rows = i1 - i0 + 1;
+    for (int t = threadIdx.x; t < num_rows * num_m; t += blockDim.x) {
+      const int i = i0 + t / num_m;
+      const int m = m_first + t % num_m;
+      const int j_lo = (i == i0) ? q0 - i * sk : 0;
+      const int j_hi = (i == i1) ? q1 - i * sk : sk - 1;
+      const int sm = g.side[m];
+      const int r = (m == q_scale) ? r_own : r_prev;
+      const int ci = static_cast<int>((static_cast<int64_t>(i) * sm) / sk);
+      const int cl = static_cast<int>((static_cast<int64_t>(j_lo) * sm) / sk);
+      const int ch = static_cast<int>((static_cast<int64_t>(j_hi) * sm) / sk);
+      const int a_lo = max(0, ci - r), a_hi = min(sm - 1, ci + r);
+      const int b_lo = max(0, cl - r), b_hi = min(sm - 1, ch + r);
+      for (int a = a_lo; a <= a_hi; ++a) {
+        const int t_lo = g.off[m] + a * sm + b_lo;
+        const int t_hi = g.off[m] + a * sm + b_hi;
+        set_bit_range(bits, t_lo / block_kv, t_hi / block_kv);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 32)
+    compact_bitset(bits, nkb, kv_idx + static_cast<int64_t>(qb) * nkb, kv_cnt + qb,
+                   blk_mask ? blk_mask + static_cast<int64_t>(qb) * nkb : nullptr);
+}
+
+// ---------------------------------------------------------------- CS4A mapping
+__device__ __forceinline__ int64_t floor_scale(int64_t x, int64_t num, int64_t den) {
+  return (x * num) / den;
+}
+__device__ __forceinline__ int64_t ceil_scale(int64_t x, int64_t num, int64_t den) {
+  return (x * num + den - 1) / den;
+}
+
+__global__ void __launch_bounds__(kMaskThreads)
+    map_indices_kernel(const int32_t* src_cnt, const int32_t* src_idx, int H, int s_nq,
+                       int s_lkv, int d_nq, int d_lkv, int block_q, int block_kv, int s_nqb,
+                       int s_nkb, int d_nqb, int d_nkb, int n_sink_tok, int32_t* d_cnt,
+                       int32_t* d_idx, uint8_t* d_mask, int32_t* dev_status) {
+  extern __shared__ uint32_t bits[];
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  const int nwords = (d_nkb + 31) >> 5;
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bits[w] = 0u;
+  __syncthreads();
+
+  const int a = qb * block_q;
+  const int bnd = min(a + block_q, d_nq);
+  for (int t = threadIdx.x; t < s_nqb * s_nkb; t += blockDim.x) {
+    const int qs = t / s_nkb, e = t % s_nkb;
+    const int64_t srow = bh * s_nqb + qs;
+    int cnt = src_cnt[srow];
+    if (cnt < 0 || cnt > s_nkb) {
+      if (e == 0 && dev_status) atomicOr(dev_status, 0x1);
+      cnt = cnt < 0 ? 0 : s_nkb;
+    }
+    if (e >= cnt) continue;
+    const int qlo = qs * block_q, qhi = min(qlo + block_q, s_nq);
+    const int64_t tq_lo = floor_scale(qlo, d_nq, s_nq);
+    const int64_t tq_hi = ceil_scale(qhi, d_nq, s_nq);
+    if (!(a < tq_hi && tq_lo < bnd)) continue;
+    const int kb = src_idx[srow * s_nkb + e];
+    if (kb < 0 || kb >= s_nkb) {
+      if (dev_status) atomicOr(dev_status, 0x1);
+      continue;
+    }
+    const int klo = kb * block_kv, khi = min(klo + block_kv, s_lkv);
+    const int64_t tk_lo = floor_scale(klo, d_lkv, s_lkv);
+    const int64_t tk_hi = min(ceil_scale(khi, d_lkv, s_lkv), static_cast<int64_t>(d_lkv));
+    if (tk_hi > tk_lo)
+      set_bit_range(bits, static_cast<int>(tk_lo / block_kv),
+                    static_cast<int>((tk_hi - 1) / block_kv));
+  }
+  if (threadIdx.x == 0 && n_sink_tok > 0)
+    set_bit_range(bits, 0, min(d_nkb - 1, (n_sink_tok - 1) / block_kv));
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int64_t drow = bh * d_nqb + qb;
+    compact_bitset(bits, d_nkb, d_idx + drow * d_nkb, d_cnt + drow,
+                   d_mask ? d_mask + drow * d_nkb : nullptr);
+  }
+}
+
+// ---------------------------------------------------------------- validation
+__global__ void validate_lists_kernel(const int32_t* kv_cnt, const int32_t* kv_idx, int n_rows,
+                                      int row_len, int nkb, int32_t* dev_status) {
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  int flags = 0;
+  int cnt = kv_cnt[row];
+  if (cnt < 0 || cnt > row_len || cnt > nkb) {
+    flags |= 0x1;
+    cnt = cnt < 0 ? 0 : min(row_len, nkb);
+  }
+  const int32_t* r = kv_idx + static_cast<int64_t>(row) * row_len;
+  for (int e = lane; e < cnt; e += 32) {
+    const int v = r[e];
+    if (v < 0 || v >= nkb) flags |= 0x1;
+    if (e > 0 && r[e - 1] >= v) flags |= 0x4;
+  }
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if (lane == 0 && flags) atomicOr(dev_status, flags);
+}
+
+}  // namespace sparvar

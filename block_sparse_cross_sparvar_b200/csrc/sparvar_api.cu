@@ -1,0 +1,326 @@
+// C-ABI entry points of libsparvar.so (declared in include/sparvar.h).
+// Host-side argument checks, TMA tensor-map encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/sparvar.h"
+#include "attn_kernel.cuh"
+#include "mask_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SPARVAR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool block_ok(int b) { return b == 16 || b == 32 || b == 64 || b == 128; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int build_geometry(const int32_t* sides, int n_scales, sparvar::ScaleGeometry* g) {
+  if (!sides) return fail(SPARVAR_ERR_INVALID_ARG, "sides is NULL");
+  if (n_scales < 1 || n_scales > SPARVAR_MAX_SCALES)
+    return fail(SPARVAR_ERR_INVALID_ARG, "n_scales=%d outside [1, %d]", n_scales,
+                SPARVAR_MAX_SCALES);
+  g->n_scales = n_scales;
+  int64_t off = 0;
+  g->off[0] = 0;
+  for (int m = 0; m < n_scales; ++m) {
+    if (sides[m] < 1 || sides[m] > 46340)
+      return fail(SPARVAR_ERR_INVALID_ARG, "sides[%d]=%d outside [1, 46340]", m, sides[m]);
+    g->side[m] = sides[m];
+    off += static_cast<int64_t>(sides[m]) * sides[m];
+    if (off > (1ll << 30)) return fail(SPARVAR_ERR_INVALID_ARG, "total tokens exceed 2^30");
+    g->off[m + 1] = static_cast<int>(off);
+  }
+  return SPARVAR_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D map over a [B][H][rows][D] bf16 tensor: box = 64 columns x 128 rows,
+// 128-byte swizzle, zero fill outside the tensor.
+int make_tmap(CUtensorMap* m, const void* base, int D, int rows, int H, int B, int64_t sr,
+              int64_t sh, int64_t sb, const char* name) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(SPARVAR_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (H == 1) sh = static_cast<int64_t>(rows) * sr;
+  if (B == 1) sb = static_cast<int64_t>(H) * sh;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(sr * 2), static_cast<cuuint64_t>(sh * 2),
+                           static_cast<cuuint64_t>(sb * 2)};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(SPARVAR_ERR_INVALID_ARG, "tensor map for %s rejected (CUresult %d)", name,
+                static_cast<int>(r));
+  return SPARVAR_OK;
+}
+
+// Row stride, head stride and batch stride of one [B][H][rows][D] operand.
+int check_operand(const void* p, const int64_t* st, int B, int H, int rows, int D,
+                  const char* name) {
+  if (!p) return fail(SPARVAR_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(SPARVAR_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  if (!st) return fail(SPARVAR_ERR_INVALID_ARG, "%s strides are NULL", name);
+  const int64_t sb = st[0], sh = st[1], sr = st[2];
+  if (sr < D || (sr % 8) != 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "%s row stride %lld must be >= D and a multiple of 8",
+                name, static_cast<long long>(sr));
+  if (H > 1 && (sh <= 0 || (sh % 8) != 0))
+    return fail(SPARVAR_ERR_INVALID_ARG, "%s head stride %lld must be a positive multiple of 8",
+                name, static_cast<long long>(sh));
+  if (B > 1 && (sb <= 0 || (sb % 8) != 0))
+    return fail(SPARVAR_ERR_INVALID_ARG, "%s batch stride %lld must be a positive multiple of 8",
+                name, static_cast<long long>(sb));
+  if (sr * 2 >= (1ll << 40) || sh * 2 >= (1ll << 40) || sb * 2 >= (1ll << 40))
+    return fail(SPARVAR_ERR_INVALID_ARG, "%s strides too large", name);
+  (void)rows;
+  return SPARVAR_OK;
+}
+
+template <int D, int MODE>
+int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const sparvar::AttnArgs& a, cudaStream_t stream) {
+  auto kern = sparvar::block_sparse_attn_kernel<D, MODE>;
+  const uint32_t smem = sparvar::Smem<D>::dyn_bytes(MODE);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  dim3 grid(a.nqb, a.H, a.B);
+  kern<<<grid, sparvar::kThreads, smem, stream>>>(tq, tk, tv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block_sparse_attn_kernel launch");
+  return SPARVAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sparvar_last_error(void) { return g_last_error.c_str(); }
+
+const char* sparvar_version(void) { return "sparvar-b200 0.1 (sm_100a)"; }
+
+int sparvar_scale_blocks(const int32_t* sides, int n_scales, int q_scale, int block_q,
+                         int block_kv, int32_t* nqb, int32_t* nkb) {
+  sparvar::ScaleGeometry g;
+  int rc = build_geometry(sides, n_scales, &g);
+  if (rc) return rc;
+  if (q_scale < 0 || q_scale >= n_scales)
+    return fail(SPARVAR_ERR_INVALID_ARG, "q_scale=%d outside [0, %d)", q_scale, n_scales);
+  if (block_q < 1 || block_kv < 1) return fail(SPARVAR_ERR_INVALID_ARG, "block sizes must be >= 1");
+  if (!nqb || !nkb) return fail(SPARVAR_ERR_INVALID_ARG, "output pointers are NULL");
+  const int64_t nq = static_cast<int64_t>(g.side[q_scale]) * g.side[q_scale];
+  *nqb = static_cast<int32_t>(ceil_div(nq, block_q));
+  *nkb = static_cast<int32_t>(ceil_div(g.off[q_scale + 1], block_kv));
+  return SPARVAR_OK;
+}
+
+int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int q_scale, int n_sink_scales,
+                            int radius_prev, int radius_own, int block_q, int block_kv,
+                            int32_t* kv_cnt, int32_t* kv_idx, uint8_t* blk_mask, void* stream) {
+  sparvar::ScaleGeometry g;
+  int rc = build_geometry(sides, n_scales, &g);
+  if (rc) return rc;
+  if (q_scale < 0 || q_scale >= n_scales)
+    return fail(SPARVAR_ERR_INVALID_ARG, "q_scale=%d outside [0, %d)", q_scale, n_scales);
+  if (n_sink_scales < 0) return fail(SPARVAR_ERR_INVALID_ARG, "n_sink_scales < 0");
+  if (radius_prev < 0 || radius_own < 0) return fail(SPARVAR_ERR_INVALID_ARG, "radius < 0");
+  if (!block_ok(block_q) || !block_ok(block_kv))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "block sizes (%d, %d) not in {16, 32, 64, 128}", block_q,
+                block_kv);
+  if (!kv_cnt || !kv_idx) return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx is NULL");
+  const int64_t nq = static_cast<int64_t>(g.side[q_scale]) * g.side[q_scale];
+  const int nqb = static_cast<int>(ceil_div(nq, block_q));
+  const int nkb = static_cast<int>(ceil_div(g.off[q_scale + 1], block_kv));
+  const size_t smem = static_cast<size_t>((nkb + 31) / 32) * 4;
+  if (smem > 48 * 1024) return fail(SPARVAR_ERR_UNSUPPORTED, "too many KV blocks (%d)", nkb);
+  sparvar::csla_mask_kernel<<<nqb, sparvar::kMaskThreads, smem,
+                              static_cast<cudaStream_t>(stream)>>>(
+      g, q_scale, n_sink_scales, radius_prev, radius_own, block_q, block_kv, nkb, kv_cnt, kv_idx,
+      blk_mask);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "csla_mask_kernel launch");
+  return SPARVAR_OK;
+}
+
+int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_idx, int B, int H, int src_nq,
+                        int src_lkv, int dst_nq, int dst_lkv, int block_q, int block_kv,
+                        int n_sink_tokens, int32_t* dst_cnt, int32_t* dst_idx,
+                        uint8_t* dst_blk_mask, int32_t* dev_status, void* stream) {
+  if (!src_cnt || !src_idx || !dst_cnt || !dst_idx)
+    return fail(SPARVAR_ERR_INVALID_ARG, "list pointer is NULL");
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (src_nq < 1 || src_lkv < 1 || dst_nq < 1 || dst_lkv < 1)
+    return fail(SPARVAR_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (src_nq > (1 << 30) || src_lkv > (1 << 30) || dst_nq > (1 << 30) || dst_lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "sizes must be <= 2^30");
+  if (!block_ok(block_q) || !block_ok(block_kv))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "block sizes (%d, %d) not in {16, 32, 64, 128}", block_q,
+                block_kv);
+  if (n_sink_tokens < 0) return fail(SPARVAR_ERR_INVALID_ARG, "n_sink_tokens < 0");
+  const int s_nqb = static_cast<int>(ceil_div(src_nq, block_q));
+  const int s_nkb = static_cast<int>(ceil_div(src_lkv, block_kv));
+  const int d_nqb = static_cast<int>(ceil_div(dst_nq, block_q));
+  const int d_nkb = static_cast<int>(ceil_div(dst_lkv, block_kv));
+  const size_t smem = static_cast<size_t>((d_nkb + 31) / 32) * 4;
+  if (smem > 48 * 1024) return fail(SPARVAR_ERR_UNSUPPORTED, "too many KV blocks (%d)", d_nkb);
+  if (static_cast<int64_t>(s_nqb) * s_nkb > (1ll << 30))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "source block grid too large");
+  dim3 grid(d_nqb, H, B);
+  sparvar::map_indices_kernel<<<grid, sparvar::kMaskThreads, smem,
+                                static_cast<cudaStream_t>(stream)>>>(
+      src_cnt, src_idx, H, src_nq, src_lkv, dst_nq, dst_lkv, block_q, block_kv, s_nqb, s_nkb,
+      d_nqb, d_nkb, n_sink_tokens, dst_cnt, dst_idx, dst_blk_mask, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "map_indices_kernel launch");
+  return SPARVAR_OK;
+}
+
+int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_rows,
+                           int idx_row_len, int nkb, int32_t* dev_status, void* stream) {
+  if (!kv_cnt || !kv_idx || !dev_status)
+    return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx/dev_status is NULL");
+  if (n_rows < 0 || idx_row_len < 0 || nkb < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "negative size");
+  if (n_rows == 0) return SPARVAR_OK;
+  const int warps = 8;
+  sparvar::validate_lists_kernel<<<static_cast<unsigned>(ceil_div(n_rows, warps)), warps * 32, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(
+      kv_cnt, kv_idx, n_rows, idx_row_len, nkb, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "validate_lists_kernel launch");
+  return SPARVAR_OK;
+}
+
+int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int H, int Lq, int Lkv, int D,
+                                  const int64_t* q_strides, const int64_t* k_strides,
+                                  const int64_t* v_strides, const int64_t* o_strides,
+                                  const int32_t* kv_cnt, const int32_t* kv_idx,
+                                  const int64_t* list_strides, int idx_row_len, int block_q,
+                                  int block_kv, float softmax_scale, int32_t* dev_status,
+                                  void* stream) {
+  if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
+  if (block_q != 128 || block_kv != 128)
+    return fail(SPARVAR_ERR_UNSUPPORTED,
+                "attention blocks (%d, %d): this kernel takes 128 x 128 blocks", block_q,
+                block_kv);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  int rc;
+  if ((rc = check_operand(q, q_strides, B, H, Lq, D, "q"))) return rc;
+  if ((rc = check_operand(k, k_strides, B, H, Lkv, D, "k"))) return rc;
+  if ((rc = check_operand(v, v_strides, B, H, Lkv, D, "v"))) return rc;
+  if ((rc = check_operand(o, o_strides, B, H, Lq, D, "o"))) return rc;
+  if (!kv_cnt || !kv_idx || !list_strides)
+    return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx/list_strides is NULL");
+  if (list_strides[0] < 0 || list_strides[1] < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
+  if (idx_row_len < 0) return fail(SPARVAR_ERR_INVALID_ARG, "idx_row_len < 0");
+  if (!std::isfinite(softmax_scale)) return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale not finite");
+
+  sparvar::AttnArgs a{};
+  a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
+  a.nqb = static_cast<int>(ceil_div(Lq, 128));
+  a.nkb = static_cast<int>(ceil_div(Lkv, 128));
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.kv_cnt = kv_cnt; a.kv_idx = kv_idx;
+  a.list_sb = list_strides[0]; a.list_sh = list_strides[1];
+  a.idx_row_len = idx_row_len;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
+  a.lse_out = lse;
+  a.dev_status = dev_status;
+
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
+  if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
+  if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return launch_attn_kernel<128, sparvar::kModeAttn>(tq, tk, tv, a, st);
+  return launch_attn_kernel<64, sparvar::kModeAttn>(tq, tk, tv, a, st);
+}
+
+int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
+                          const int64_t* q_strides, const int64_t* k_strides, float softmax_scale,
+                          const float* lse, int block_q, int block_kv, float mass_threshold,
+                          int32_t* kv_cnt, int32_t* kv_idx, float* mass, int32_t* dev_status,
+                          void* stream) {
+  if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
+  if (block_q != 128 || block_kv != 128)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "decision blocks (%d, %d): 128 x 128 only", block_q,
+                block_kv);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  const int nkb = static_cast<int>(ceil_div(Lkv, 128));
+  if (nkb > sparvar::kMaxMassBlocks)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "Lkv=%d gives %d KV blocks (max %d)", Lkv, nkb,
+                sparvar::kMaxMassBlocks);
+  int rc;
+  if ((rc = check_operand(q, q_strides, B, H, Lq, D, "q"))) return rc;
+  if ((rc = check_operand(k, k_strides, B, H, Lkv, D, "k"))) return rc;
+  if (!kv_cnt || !kv_idx) return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx is NULL");
+  if (!std::isfinite(softmax_scale) || std::isnan(mass_threshold))
+    return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale or mass_threshold not a number");
+
+  sparvar::AttnArgs a{};
+  a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
+  a.nqb = static_cast<int>(ceil_div(Lq, 128));
+  a.nkb = nkb;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.lse_in = lse;
+  a.mass_threshold = mass_threshold;
+  a.sel_cnt = kv_cnt; a.sel_idx = kv_idx; a.mass_out = mass;
+  a.dev_status = dev_status;
+  CUtensorMap tq, tk;
+  if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
+  if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return launch_attn_kernel<128, sparvar::kModeMass>(tq, tk, tk, a, st);
+  return launch_attn_kernel<64, sparvar::kModeMass>(tq, tk, tk, a, st);
+}
+
+}  // extern "C"

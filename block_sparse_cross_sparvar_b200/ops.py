@@ -1,0 +1,213 @@
+"""Python binding of libsparvar.so: the C-ABI calls under the same names.
+
+Argument marshalling only: tensors are allocated by torch (device memory,
+current stream), every step of the computation runs in the library's CUDA
+kernels.  A missing library raises immediately; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsparvar.so")
+
+SPARVAR_DEV_BAD_LIST = 0x1
+SPARVAR_DEV_TIMEOUT = 0x2
+SPARVAR_DEV_NOT_ASCENDING = 0x4
+
+_lib = None
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+EXPORTS = {
+    "sparvar_last_error": ([], ctypes.c_char_p),
+    "sparvar_version": ([], ctypes.c_char_p),
+    "sparvar_scale_blocks": ([_i32p, _i, _i, _i, _i, _i32p, _i32p], _i),
+    "sparvar_build_csla_mask": ([_i32p, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
+    "sparvar_decide_blocks": ([_vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p, _f, _vp, _i, _i, _f,
+                               _vp, _vp, _vp, _vp, _vp], _i),
+    "sparvar_map_indices": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                             _vp], _i),
+    "sparvar_block_sparse_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p,
+                                       _i64p, _i64p, _vp, _vp, _i64p, _i, _i, _i, _f, _vp, _vp],
+                                      _i),
+    "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
+}
+
+
+class SparvarError(RuntimeError):
+    pass
+
+
+def lib():
+    """Load libsparvar.so (built in-tree) and declare its signatures."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise SparvarError(
+                f"{LIB_PATH} is missing: build it with `python -m block_sparse_cross_sparvar_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in EXPORTS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def _check(rc: int, name: str):
+    if rc != 0:
+        msg = lib().sparvar_last_error().decode()
+        raise SparvarError(f"{name} failed (status {rc}): {msg}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _i64(vals):
+    return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _bhrd(t, name):
+    if t.dim() != 4:
+        raise SparvarError(f"{name} must be [B, H, rows, D], got {tuple(t.shape)}")
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise SparvarError(f"{name} must be a CUDA bf16 tensor")
+    if t.stride(3) != 1:
+        raise SparvarError(f"{name} must have a contiguous last dimension")
+    return _i64([t.stride(0), t.stride(1), t.stride(2)])
+
+
+def scale_blocks(sides, q_scale, block_q, block_kv):
+    arr = (ctypes.c_int32 * len(sides))(*sides)
+    nqb, nkb = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().sparvar_scale_blocks(arr, len(sides), q_scale, block_q, block_kv,
+                                      ctypes.byref(nqb), ctypes.byref(nkb)), "sparvar_scale_blocks")
+    return nqb.value, nkb.value
+
+
+def sparvar_build_csla_mask(sides, q_scale, n_sink_scales, radius_prev, radius_own,
+                            block_q=128, block_kv=128, device="cuda", with_mask=False):
+    """CSLA block lists for one query scale: (kv_cnt [NQB], kv_idx [NQB, NKB], blk_mask|None)."""
+    nqb, nkb = scale_blocks(sides, q_scale, block_q, block_kv)
+    cnt = torch.empty(nqb, dtype=torch.int32, device=device)
+    idx = torch.empty(nqb, nkb, dtype=torch.int32, device=device)
+    mask = torch.empty(nqb, nkb, dtype=torch.uint8, device=device) if with_mask else None
+    arr = (ctypes.c_int32 * len(sides))(*sides)
+    _check(lib().sparvar_build_csla_mask(arr, len(sides), q_scale, n_sink_scales, radius_prev,
+                                         radius_own, block_q, block_kv, _ptr(cnt), _ptr(idx),
+                                         _ptr(mask), _stream(cnt.device)), "sparvar_build_csla_mask")
+    return cnt, idx, mask
+
+
+def _list_strides(kv_cnt, B, H):
+    """List-row strides (b, h) for counts shaped [NQB], [H, NQB] or [B, H, NQB]."""
+    if not kv_cnt.is_contiguous():
+        raise SparvarError("kv_cnt must be contiguous")
+    nqb = kv_cnt.shape[-1]
+    if kv_cnt.dim() == 1:
+        return (0, 0)
+    if kv_cnt.dim() == 2:
+        if kv_cnt.shape[0] not in (1, H):
+            raise SparvarError("kv_cnt [H, NQB] does not match H")
+        return (0, nqb if kv_cnt.shape[0] == H else 0)
+    if kv_cnt.dim() == 3:
+        if kv_cnt.shape[0] not in (1, B) or kv_cnt.shape[1] not in (1, H):
+            raise SparvarError("kv_cnt [B, H, NQB] does not match B, H")
+        sh = nqb if kv_cnt.shape[1] == H else 0
+        sb = kv_cnt.shape[1] * nqb if kv_cnt.shape[0] == B else 0
+        return (sb, sh)
+    raise SparvarError("kv_cnt must be 1-, 2- or 3-D")
+
+
+def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv=128,
+                                  softmax_scale=None, out=None, return_lse=False, dev_status=None):
+    """Block-sparse attention forward: returns O (and the row LSE when asked)."""
+    B, H, Lq, D = q.shape
+    Lkv = k.shape[2]
+    if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
+        raise SparvarError("k/v must be [B, H, Lkv, D] matching q")
+    qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    os_ = _bhrd(out, "out")
+    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32:
+        raise SparvarError("kv_cnt/kv_idx must be int32")
+    if kv_idx.shape[:-1] != kv_cnt.shape or not kv_idx.is_contiguous():
+        raise SparvarError("kv_idx must be contiguous with shape (*kv_cnt.shape, row_len)")
+    nqb = -(-Lq // block_q)
+    if kv_cnt.shape[-1] != nqb:
+        raise SparvarError(f"kv_cnt has {kv_cnt.shape[-1]} query blocks, expected {nqb}")
+    lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    sb, sh = _list_strides(kv_cnt, B, H)
+    _check(lib().sparvar_block_sparse_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
+        _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], block_q, block_kv, scale,
+        _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sparvar_decide_blocks(q, k, mass_threshold, lse=None, softmax_scale=None, block_q=128,
+                          block_kv=128, return_mass=False, dev_status=None):
+    """CS4A decision: (kv_cnt [B,H,NQB], kv_idx [B,H,NQB,NKB], mass|None)."""
+    B, H, Lq, D = q.shape
+    Lkv = k.shape[2]
+    qs, ks = _bhrd(q, "q"), _bhrd(k, "k")
+    nqb, nkb = -(-Lq // block_q), -(-Lkv // block_kv)
+    cnt = torch.empty(B, H, nqb, dtype=torch.int32, device=q.device)
+    idx = torch.empty(B, H, nqb, nkb, dtype=torch.int32, device=q.device)
+    mass = torch.empty(B, H, nqb, nkb, dtype=torch.float32, device=q.device) if return_mass else None
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or lse.shape != (B, H, Lq)):
+        raise SparvarError("lse must be contiguous fp32 [B, H, Lq]")
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    _check(lib().sparvar_decide_blocks(
+        _ptr(q), _ptr(k), B, H, Lq, Lkv, D, qs, ks, scale, _ptr(lse), block_q, block_kv,
+        float(mass_threshold), _ptr(cnt), _ptr(idx), _ptr(mass), _ptr(dev_status),
+        _stream(q.device)), "sparvar_decide_blocks")
+    return cnt, idx, mass
+
+
+def sparvar_map_indices(src_cnt, src_idx, src_nq, src_lkv, dst_nq, dst_lkv, block_q=128,
+                        block_kv=128, n_sink_tokens=0, with_mask=False, dev_status=None):
+    """CS4A mapping of [B, H, NQB_src] lists onto a later scale: (cnt, idx, mask|None)."""
+    if src_cnt.dim() != 3 or not src_cnt.is_contiguous() or not src_idx.is_contiguous():
+        raise SparvarError("src_cnt must be contiguous [B, H, NQB_src]; src_idx contiguous")
+    B, H, s_nqb = src_cnt.shape
+    s_nkb = -(-src_lkv // block_kv)
+    if src_idx.shape != (B, H, s_nqb, s_nkb):
+        raise SparvarError(f"src_idx must be [B, H, {s_nqb}, {s_nkb}]")
+    d_nqb, d_nkb = -(-dst_nq // block_q), -(-dst_lkv // block_kv)
+    dev = src_cnt.device
+    cnt = torch.empty(B, H, d_nqb, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, H, d_nqb, d_nkb, dtype=torch.int32, device=dev)
+    mask = torch.empty(B, H, d_nqb, d_nkb, dtype=torch.uint8, device=dev) if with_mask else None
+    _check(lib().sparvar_map_indices(
+        _ptr(src_cnt), _ptr(src_idx), B, H, src_nq, src_lkv, dst_nq, dst_lkv, block_q, block_kv,
+        n_sink_tokens, _ptr(cnt), _ptr(idx), _ptr(mask), _ptr(dev_status), _stream(dev)),
+        "sparvar_map_indices")
+    return cnt, idx, mask
+
+
+def sparvar_validate_lists(kv_cnt, kv_idx, nkb):
+    """Device check of lists; returns the SPARVAR_DEV_* bits found (synchronises)."""
+    status = torch.zeros(1, dtype=torch.int32, device=kv_cnt.device)
+    n_rows = kv_cnt.numel()
+    _check(lib().sparvar_validate_lists(_ptr(kv_cnt), _ptr(kv_idx), n_rows, kv_idx.shape[-1], nkb,
+                                        _ptr(status), _stream(kv_cnt.device)),
+           "sparvar_validate_lists")
+    return int(status.item())

@@ -1,0 +1,207 @@
+/*
+ * sparvar.h - C ABI of libsparvar.so: block-sparse cross-scale attention for
+ * next-scale-prediction (VAR) transformers on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the SparVAR pages ("SparVAR: Exploring Sparsity in
+ * Visual AutoRegressive Modeling for Training-Free Acceleration", ai.info
+ * summary): section "Methodology in Plain English" defines CSLA (sink +
+ * cross-scale locality mask aggregated into blocks) and CS4A (block pooling
+ * of dense attention at a sparse decision scale, top-block selection, index
+ * rescaling to later scales); sections "Key Contributions" (item 3) and
+ * "Main Findings" (block sizes 64/128) define the block-wise sparse kernel;
+ * section "What This Paper Is About" fixes that a scale's queries attend to
+ * all tokens of all earlier scales and of their own scale.
+ *
+ * Conventions shared by every call
+ *  - Scales are square; scale m (0-based) has side sides[m] and holds tokens
+ *    [off[m], off[m+1]) of the concatenated sequence, off[m] = sum_{i<m} side_i^2,
+ *    row-major inside a scale.
+ *  - Query blocks are numbered locally inside the query scale: qb covers query
+ *    rows [qb*block_q, min((qb+1)*block_q, Lq)).  KV blocks are numbered
+ *    globally over the key prefix: kb covers keys [kb*block_kv, min(.., Lkv)).
+ *  - A block list for one query block is an int32 count plus an int32 row of
+ *    KV-block indices; the first `count` entries are used.  Lists written by
+ *    this library are ascending and padded with -1.
+ *  - Tensors are bf16, laid out [B][H][rows][D] with arbitrary element strides
+ *    for B, H and rows and a contiguous last dimension.
+ *  - Device pointers are plain CUDA device addresses; "host" marks the few
+ *    arguments read from host memory during the call.
+ *  - The caller allocates and owns every buffer.  Calls enqueue work on
+ *    `stream` (a cudaStream_t; NULL = legacy default stream), never
+ *    synchronise, and never allocate device memory.
+ *  - Every call returns a sparvar_status.  Arguments are checked on the host
+ *    before anything is enqueued; on failure nothing is enqueued and
+ *    sparvar_last_error() describes the problem.  Problems that can only be
+ *    seen on the device (a list entry out of range, a bounded wait that gave
+ *    up) are OR-ed into the optional `dev_status` word as SPARVAR_DEV_* bits;
+ *    kernels never trap.
+ */
+#ifndef SPARVAR_H_
+#define SPARVAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPARVAR_API __attribute__((visibility("default")))
+#else
+#define SPARVAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPARVAR_OK = 0,
+  SPARVAR_ERR_INVALID_ARG = 1,  /* bad pointer, size, stride or alignment      */
+  SPARVAR_ERR_UNSUPPORTED = 2,  /* valid request outside what is implemented  */
+  SPARVAR_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed           */
+} sparvar_status;
+
+/* Bits OR-ed into *dev_status by kernels. */
+#define SPARVAR_DEV_BAD_LIST 0x1 /* count < 0, count > row length, or an index outside [0, nkb) */
+#define SPARVAR_DEV_TIMEOUT 0x2  /* a bounded wait inside a kernel gave up; outputs are invalid  */
+#define SPARVAR_DEV_NOT_ASCENDING 0x4 /* (validate only) indices not strictly ascending   */
+
+#define SPARVAR_MAX_SCALES 32
+
+/* Thread-local description of the last failing call on this thread. */
+SPARVAR_API const char* sparvar_last_error(void);
+
+/* Library version string. */
+SPARVAR_API const char* sparvar_version(void);
+
+/*
+ * Number of query blocks and KV blocks for query scale `q_scale`:
+ *   *nqb = ceil(sides[q_scale]^2 / block_q), *nkb = ceil(off[q_scale+1] / block_kv).
+ * sides: host array of n_scales side lengths.  Pure host computation.
+ */
+SPARVAR_API int sparvar_scale_blocks(const int32_t* sides, int n_scales, int q_scale, int block_q,
+                         int block_kv, int32_t* nqb, int32_t* nkb);
+
+/*
+ * CSLA block mask for the queries of scale `q_scale`
+ * ("Methodology in Plain English", CSLA paragraph; sinks and windows from
+ * "Main Findings").
+ *
+ * Token rule: query (i, j) of the side-s_k query scale keeps key token t when
+ *   t < off[n_sink_scales]                                   (sink prior), or
+ *   t lies in scale m, n_sink_scales <= m <= q_scale, at (a, b), with
+ *   max(|a - floor(i*s_m/s_k)|, |b - floor(j*s_m/s_k)|) <= r_m, where
+ *   r_m = radius_own if m == q_scale else radius_prev   (locality prior).
+ * A (query block, KV block) is kept when any of its token pairs is kept.
+ * The mask depends only on the geometry, so one list serves every batch item
+ * and head (pass zero list strides to the attention call).
+ *
+ * sides      host, n_scales int32 side lengths (1 <= n_scales <= SPARVAR_MAX_SCALES).
+ * block_q, block_kv  in {16, 32, 64, 128}.
+ * kv_cnt     device, int32[nqb]          out: kept KV blocks per query block.
+ * kv_idx     device, int32[nqb * nkb]    out: ascending kept indices, -1 padded.
+ * blk_mask   device, uint8[nqb * nkb] or NULL; out: 1 = kept.
+ */
+SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int q_scale,
+                            int n_sink_scales, int radius_prev, int radius_own,
+                            int block_q, int block_kv, int32_t* kv_cnt, int32_t* kv_idx,
+                            uint8_t* blk_mask, void* stream);
+
+/*
+ * CS4A decision: pooled softmax mass of dense attention at the sparse decision
+ * scale and per-query-block selection ("Methodology in Plain English", CS4A
+ * paragraph: split the dense map into query blocks, sum the attention weights
+ * in each block, keep the top blocks; decision scale from "Main Findings").
+ *
+ *   mass[qb, kb] = (1 / n_q(qb)) * sum_{q in qb} sum_{key in kb} exp(s(q,key) - lse(q)),
+ *   s = softmax_scale * q . key over all Lkv keys (no mask), lse = log-sum-exp of row q.
+ * Per query block, KV blocks are ordered by mass (descending, ties to the lower
+ * index) and the shortest prefix whose running sum reaches mass_threshold is
+ * kept (every block when the total stays below it).  Kept lists are written in
+ * ascending order.
+ *
+ * q [B][H][Lq][D], k [B][H][Lkv][D]: device bf16; strides in elements for
+ *   (b, h, row) given by host arrays q_strides[3], k_strides[3]; row strides and
+ *   base addresses 16-byte aligned; D in {64, 128}.
+ * lse        device fp32 [B][H][Lq] contiguous (natural log), or NULL to have the
+ *            call compute it (one extra sweep over the keys).
+ * block_q = block_kv = 128.
+ * kv_cnt     device int32 [B][H][nqb]; kv_idx device int32 [B][H][nqb][nkb] (-1 padded).
+ * mass       device fp32 [B][H][nqb][nkb] or NULL.
+ * dev_status device int32 or NULL.
+ */
+SPARVAR_API int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
+                          const int64_t* q_strides, const int64_t* k_strides,
+                          float softmax_scale, const float* lse, int block_q, int block_kv,
+                          float mass_threshold, int32_t* kv_cnt, int32_t* kv_idx, float* mass,
+                          int32_t* dev_status, void* stream);
+
+/*
+ * CS4A cross-scale index mapping ("Methodology in Plain English", CS4A
+ * paragraph: kept positions are rescaled to a later, larger scale, optionally
+ * adding the sink region).
+ *
+ * A kept source block covering query rows [qlo, qhi) and keys [klo, khi) covers
+ * destination query rows [floor(qlo*dst_nq/src_nq), ceil(qhi*dst_nq/src_nq)) and
+ * keys [floor(klo*dst_lkv/src_lkv), ceil(khi*dst_lkv/src_lkv)); every destination
+ * block meeting both ranges is kept.  The union over all kept source blocks is
+ * taken, and every destination KV block holding a key < n_sink_tokens is kept in
+ * every row.
+ *
+ * src_cnt  device int32 [B][H][src_nqb]; src_idx device int32 [B][H][src_nqb][src_nkb]
+ *          (src_nqb = ceil(src_nq/block_q), src_nkb = ceil(src_lkv/block_kv)).
+ * dst_cnt  device int32 [B][H][dst_nqb]; dst_idx device int32 [B][H][dst_nqb][dst_nkb].
+ * dst_blk_mask device uint8 [B][H][dst_nqb][dst_nkb] or NULL.
+ * block_q, block_kv in {16, 32, 64, 128}.  dev_status device int32 or NULL
+ * (SPARVAR_DEV_BAD_LIST for source entries out of range; they are skipped).
+ */
+SPARVAR_API int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_idx, int B, int H,
+                        int src_nq, int src_lkv, int dst_nq, int dst_lkv, int block_q,
+                        int block_kv, int n_sink_tokens, int32_t* dst_cnt, int32_t* dst_idx,
+                        uint8_t* dst_blk_mask, int32_t* dev_status, void* stream);
+
+/*
+ * Block-sparse attention forward ("Key Contributions" item 3, "Main
+ * Findings" block-size rows; scale-causal prefix from "What This Paper Is
+ * About"):
+ *
+ *   O[q] = sum_key softmax_key(s(q,key)) V[key],  s = softmax_scale * Q[q].K[key],
+ *   keys restricted to the KV blocks listed for q's query block (dense inside a
+ *   block, key < Lkv).  A row with an empty list gives O = 0 and lse = -inf.
+ *
+ * q [B][H][Lq][D], k and v [B][H][Lkv][D], o [B][H][Lq][D]: device bf16, strides in
+ *   elements for (b, h, row) from host arrays *_strides[3]; last dim contiguous;
+ *   base addresses and row strides 16-byte aligned.  D in {64, 128}.
+ * lse        device fp32 [B][H][Lq] contiguous (natural log) or NULL.
+ * kv_cnt     device int32; the count of (b, h, qb) is at
+ *            kv_cnt[b*list_strides[0] + h*list_strides[1] + qb].
+ * kv_idx     device int32; its list is the idx_row_len entries starting at
+ *            kv_idx[(b*list_strides[0] + h*list_strides[1] + qb) * idx_row_len].
+ *            list_strides (host, 2 values, in list rows) may be 0 to share one
+ *            list set across batch items or heads.
+ * block_q = block_kv = 128.
+ * dev_status device int32 or NULL: SPARVAR_DEV_BAD_LIST when an entry is out of
+ *            range (the entry contributes nothing), SPARVAR_DEV_TIMEOUT when a
+ *            bounded wait gave up.
+ */
+SPARVAR_API int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int H, int Lq, int Lkv, int D,
+                                  const int64_t* q_strides, const int64_t* k_strides,
+                                  const int64_t* v_strides, const int64_t* o_strides,
+                                  const int32_t* kv_cnt, const int32_t* kv_idx,
+                                  const int64_t* list_strides, int idx_row_len, int block_q,
+                                  int block_kv, float softmax_scale, int32_t* dev_status,
+                                  void* stream);
+
+/*
+ * Device-side check of block lists: for each of n_rows rows,
+ * 0 <= cnt <= min(idx_row_len, nkb), entries in [0, nkb) and strictly ascending.
+ * ORs SPARVAR_DEV_BAD_LIST / SPARVAR_DEV_NOT_ASCENDING into *dev_status (required).
+ * kv_cnt int32[n_rows], kv_idx int32[n_rows * idx_row_len], both device.
+ */
+SPARVAR_API int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_rows,
+                           int idx_row_len, int nkb, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARVAR_H_ */

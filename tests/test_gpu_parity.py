@@ -1,0 +1,323 @@
+"""CUDA path vs the CPU fp64 oracle, through the C-ABI (needs a B200).
+
+Masks and index lists must match bit-exactly (the CS4A selection under the
+margin rule: rows whose decision sits within 1e-4 of a flip are checked for
+validity instead).  Attention outputs must match with max-abs <= 2e-2 and
+mean-abs <= 2e-3 against fp64 on the same bf16 inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_cross_sparvar_b200 import inputs, ops
+from oracle import sparvar_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+INF = inputs.INFINITY_SIDES
+TINY = inputs.TINY_SIDES
+
+
+def _dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# ------------------------------------------------------------------ CSLA masks
+MASK_CASES = [
+    (TINY, 4, 2, 1, 1, 16, 16),
+    (TINY, 3, 2, 1, 1, 16, 16),
+    (TINY, 4, 2, 1, 1, 128, 128),
+    (INF, 12, 5, 2, 4, 128, 128),
+    (INF, 11, 5, 2, 4, 128, 128),
+    (INF, 10, 5, 2, 4, 128, 128),
+    (INF, 12, 5, 1, 4, 128, 128),
+    (INF, 12, 5, 4, 4, 128, 128),
+    (INF, 11, 5, 1, 4, 128, 128),
+    (INF, 11, 5, 4, 4, 128, 128),
+    (INF, 12, 5, 2, 4, 64, 64),
+    (INF, 12, 8, 2, 4, 128, 128),
+    (INF, 12, 5, 3, 5, 32, 16),
+    (INF, 3, 5, 2, 4, 16, 16),
+    ((1, 3, 5, 7, 11), 4, 1, 1, 2, 16, 32),
+]
+
+
+@pytest.mark.parametrize("case", MASK_CASES, ids=lambda c: "-".join(map(str, c[1:])))
+def test_csla_mask_bit_exact(case):
+    sides, k, ns, rp, ro, bq, bk = case
+    cnt, idx, mask = ops.sparvar_build_csla_mask(sides, k, ns, rp, ro, bq, bk, with_mask=True)
+    ocnt, oidx, oblk = orc.build_csla_mask(sides, k, ns, rp, ro, bq, bk)
+    assert np.array_equal(cnt.cpu().numpy(), ocnt)
+    assert np.array_equal(idx.cpu().numpy(), oidx)
+    assert np.array_equal(mask.cpu().numpy().astype(bool), oblk)
+
+
+def test_csla_every_scale_and_block_size():
+    for bq in (16, 32, 64, 128):
+        for k in range(len(INF)):
+            cnt, idx, _ = ops.sparvar_build_csla_mask(INF, k, 5, 2, 4, bq, bq)
+            ocnt, oidx, _ = orc.build_csla_mask(INF, k, 5, 2, 4, bq, bq)
+            assert np.array_equal(cnt.cpu().numpy(), ocnt), (bq, k)
+            assert np.array_equal(idx.cpu().numpy(), oidx), (bq, k)
+
+
+# ------------------------------------------------------------------ attention
+def _check_attention(q_bits, k_bits, v_bits, blk_lists, bq, bk, D, lse_check=True, scale=None):
+    """q/k/v bits [B,H,*,D]; blk_lists = (cnt, idx) torch (shared or per (b,h))."""
+    B, H, Lq, _ = q_bits.shape
+    Lkv = k_bits.shape[2]
+    q, k, v = _dev(q_bits), _dev(k_bits), _dev(v_bits)
+    cnt, idx = blk_lists
+    st = _status()
+    o, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, bq, bk, softmax_scale=scale,
+                                               return_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    cnt_np, idx_np = cnt.cpu().numpy(), idx.cpu().numpy()
+    nkb = -(-Lkv // bk)
+    worst = 0.0
+    for b in range(B):
+        for h in range(H):
+            if cnt_np.ndim == 1:
+                c, ix = cnt_np, idx_np
+            else:
+                c, ix = cnt_np[b, h], idx_np[b, h]
+            blk = orc.lists_to_blocks(c, ix, nkb)
+            O, L = orc.masked_attention(q_bits_f(q_bits, b, h), q_bits_f(k_bits, b, h),
+                                        q_bits_f(v_bits, b, h), blk, bq, bk, scale=scale)
+            err = np.abs(o[b, h] - O)
+            assert err.max() <= MAX_ABS, (b, h, err.max())
+            assert err.mean() <= MEAN_ABS, (b, h, err.mean())
+            worst = max(worst, err.max())
+            if lse_check:
+                fin = np.isfinite(L)
+                assert np.array_equal(np.isfinite(lse[b, h]), fin)
+                assert np.abs(lse[b, h][fin] - L[fin]).max() < 1e-3
+    return worst
+
+
+def q_bits_f(bits, b, h):
+    return (bits[b, h].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_tiny_schedule_block128(D):
+    d = inputs.make_qkv(1, 1, 2, TINY, D, 2, pe=False)
+    off = d["offsets"]
+    k = len(TINY) - 1
+    q_bits = d["q"][:, :, off[k]:off[k + 1]]
+    kv = slice(0, off[k + 1])
+    cnt, idx, _ = ops.sparvar_build_csla_mask(TINY, k, 2, 1, 1, 128, 128)
+    _check_attention(q_bits, d["k"][:, :, kv], d["v"][:, :, kv], (cnt, idx), 128, 128, D)
+
+
+@pytest.mark.parametrize("q_scale,D", [(9, 128), (10, 128), (10, 64), (8, 128)])
+def test_attention_infinity_mid_scales(q_scale, D):
+    d = inputs.make_qkv(2, 1, 2, INF, D, 5)
+    off = d["offsets"]
+    q_bits = d["q"][:, :, off[q_scale]:off[q_scale + 1]]
+    kv = slice(0, off[q_scale + 1])
+    cnt, idx, _ = ops.sparvar_build_csla_mask(INF, q_scale, 5, 2, 4, 128, 128)
+    _check_attention(q_bits, d["k"][:, :, kv], d["v"][:, :, kv], (cnt, idx), 128, 128, D)
+
+
+def test_attention_dense_lists_and_random_lists_per_head():
+    rng = np.random.default_rng(5)
+    B, H, Lq, Lkv, D = 2, 2, 300, 777, 128
+    bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
+            for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
+    nqb, nkb = 3, 7
+    blk = rng.random((B, H, nqb, nkb)) < 0.4
+    blk[..., 0, :] = True  # one fully dense query block
+    blk[0, 0, 1, :] = False  # one empty list -> O = 0, lse = -inf
+    blk[1, 1, 2, :] = False
+    blk[1, 1, 2, 6] = True  # only the ragged last block
+    cnt = torch.from_numpy(blk.sum(-1).astype(np.int32)).cuda()
+    idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                kept = np.nonzero(blk[b, h, qb])[0]
+                idx_np[b, h, qb, :kept.size] = kept
+    idx = torch.from_numpy(idx_np).cuda()
+    _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D, scale=0.11)
+
+
+def test_attention_unordered_lists_give_same_result():
+    d = inputs.make_qkv(3, 1, 2, INF, 128, 5)
+    off = d["offsets"]
+    qk = 10
+    q = _dev(d["q"][:, :, off[qk]:off[qk + 1]])
+    k = _dev(d["k"][:, :, :off[qk + 1]])
+    v = _dev(d["v"][:, :, :off[qk + 1]])
+    cnt, idx, _ = ops.sparvar_build_csla_mask(INF, qk, 5, 2, 4, 128, 128)
+    o1 = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx)
+    rev = idx.clone()
+    for qb in range(cnt.shape[0]):
+        c = int(cnt[qb])
+        rev[qb, :c] = idx[qb, :c].flip(0)
+    o2 = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, rev)
+    assert (o1.float() - o2.float()).abs().max().item() < 2e-2
+
+
+def test_attention_bad_list_entries_flagged_not_trapped():
+    d = inputs.make_qkv(4, 1, 1, TINY, 64, 2, pe=False)
+    off = d["offsets"]
+    q = _dev(d["q"][:, :, off[4]:off[5]])
+    k = _dev(d["k"][:, :, :off[5]])
+    v = _dev(d["v"][:, :, :off[5]])
+    cnt = torch.tensor([2, 2], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[0, 99, -1], [1, -5, -1]], dtype=torch.int32, device="cuda")
+    st = _status()
+    o = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & ops.SPARVAR_DEV_BAD_LIST
+    # the valid entries alone give the same output
+    cnt1 = torch.tensor([1, 1], dtype=torch.int32, device="cuda")
+    idx1 = torch.tensor([[0, -1, -1], [1, -1, -1]], dtype=torch.int32, device="cuda")
+    o1 = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt1, idx1)
+    assert torch.equal(o, o1)
+    assert ops.sparvar_validate_lists(cnt, idx, 3) & ops.SPARVAR_DEV_BAD_LIST
+    assert ops.sparvar_validate_lists(cnt1, idx1, 3) == 0
+    bad_order = torch.tensor([[1, 0, -1], [0, 2, -1]], dtype=torch.int32, device="cuda")
+    assert ops.sparvar_validate_lists(cnt, bad_order, 3) == ops.SPARVAR_DEV_NOT_ASCENDING
+    over = torch.tensor([5, 1], dtype=torch.int32, device="cuda")
+    assert ops.sparvar_validate_lists(over, idx1, 3) & ops.SPARVAR_DEV_BAD_LIST
+
+
+def test_attention_full_size_sampled_rows():
+    """Infinity-2B last scale (B2 H16, 4096 x 10521, D128) in the bench's launch
+    configuration; sampled rows against the oracle evaluated row by row."""
+    d = inputs.make_qkv(0, 2, 16, INF, 128, 5)
+    off = d["offsets"]
+    q_bits = d["q"][:, :, off[12]:off[13]]
+    q, k, v = _dev(q_bits), _dev(d["k"]), _dev(d["v"])
+    cnt, idx, _ = ops.sparvar_build_csla_mask(INF, 12, 5, 2, 4, 128, 128)
+    st = _status()
+    o, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ocnt, oidx, blk = orc.build_csla_mask(INF, 12, 5, 2, 4, 128, 128)
+    rng = np.random.default_rng(0)
+    errs = []
+    for b, h in [(0, 0), (1, 15), (0, 7), (1, 3)]:
+        rows = np.unique(np.concatenate([rng.integers(0, 4096, 60), [0, 127, 128, 4095]]))
+        O, L = orc.masked_attention_rows(rows, q_bits_f(q_bits, b, h), q_bits_f(d["k"], b, h),
+                                         q_bits_f(d["v"], b, h), blk, 128, 128)
+        got = o[b, h, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        err = np.abs(got - O)
+        errs.append(err)
+        assert np.abs(lse[b, h, torch.from_numpy(rows).cuda()].cpu().numpy() - L).max() < 1e-3
+    err = np.concatenate(errs)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+    assert torch.isfinite(o.float()).all()
+
+
+# ------------------------------------------------------------------ CS4A
+def _decide_compare(q_bits, k_bits, tau, lse_dev=None):
+    B, H, Lq, D = q_bits.shape
+    q, k = _dev(q_bits), _dev(k_bits)
+    st = _status()
+    cnt, idx, mass = ops.sparvar_decide_blocks(q, k, tau, lse=lse_dev, return_mass=True,
+                                               dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    cnt, idx, mass = cnt.cpu().numpy(), idx.cpu().numpy(), mass.cpu().numpy()
+    n_margin = 0
+    for b in range(B):
+        for h in range(H):
+            ocnt, oidx, oblk, M, margin = orc.decide_blocks(q_bits_f(q_bits, b, h),
+                                                             q_bits_f(k_bits, b, h), 128, 128, tau)
+            assert np.abs(mass[b, h] - M).max() < 2e-5
+            for qb in range(M.shape[0]):
+                if margin[qb] > 1e-4:
+                    assert cnt[b, h, qb] == ocnt[qb]
+                    assert np.array_equal(idx[b, h, qb], oidx[qb])
+                else:
+                    n_margin += 1
+                    # within the margin: the GPU's own list must be a valid selection of its masses
+                    kept = idx[b, h, qb, :cnt[b, h, qb]]
+                    mk = mass[b, h, qb]
+                    assert mk[kept].sum() >= tau - 1e-5 or cnt[b, h, qb] == M.shape[1]
+    return n_margin
+
+
+def test_decide_blocks_decision_scale():
+    d = inputs.make_qkv(0, 1, 4, INF, 128, 5)
+    off = d["offsets"]
+    s = 9  # 32x32 decision scale
+    _decide_compare(d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]], 0.95)
+
+
+def test_decide_blocks_with_lse_from_attention():
+    d = inputs.make_qkv(1, 2, 2, INF, 128, 5)
+    off = d["offsets"]
+    s = 9
+    q = _dev(d["q"][:, :, off[s]:off[s + 1]])
+    k = _dev(d["k"][:, :, :off[s + 1]])
+    v = _dev(d["v"][:, :, :off[s + 1]])
+    nkb = -(-off[s + 1] // 128)
+    cnt = torch.full((8,), nkb, dtype=torch.int32, device="cuda")
+    idx = torch.arange(nkb, dtype=torch.int32, device="cuda").repeat(8, 1)
+    _, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True)
+    _decide_compare(d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]], 0.95, lse_dev=lse)
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.99, 2.0])
+def test_decide_blocks_thresholds_d64(tau):
+    d = inputs.make_qkv(2, 1, 2, INF, 64, 5)
+    off = d["offsets"]
+    s = 8
+    _decide_compare(d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]], tau)
+
+
+@pytest.mark.parametrize("dst_scale", [10, 11, 12])
+def test_map_indices_bit_exact(dst_scale):
+    off = inputs.token_offsets(INF)
+    rng = np.random.default_rng(dst_scale)
+    B, H = 2, 3
+    s_nq, s_lkv = 1024, off[10]
+    s_nqb, s_nkb = 8, -(-s_lkv // 128)
+    blk = rng.random((B, H, s_nqb, s_nkb)) < 0.3
+    cnt = blk.sum(-1).astype(np.int32)
+    idx = np.full((B, H, s_nqb, s_nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(s_nqb):
+                kept = np.nonzero(blk[b, h, qb])[0]
+                idx[b, h, qb, :kept.size] = kept
+    d_nq, d_lkv = INF[dst_scale] ** 2, off[dst_scale + 1]
+    st = _status()
+    dc, di, dm = ops.sparvar_map_indices(torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(),
+                                         s_nq, s_lkv, d_nq, d_lkv, 128, 128, off[5], with_mask=True,
+                                         dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for b in range(B):
+        for h in range(H):
+            oc, oi, ob = orc.map_indices(cnt[b, h], idx[b, h], s_nq, s_lkv, d_nq, d_lkv, 128, 128, off[5])
+            assert np.array_equal(dc[b, h].cpu().numpy(), oc)
+            assert np.array_equal(di[b, h].cpu().numpy(), oi)
+            assert np.array_equal(dm[b, h].cpu().numpy().astype(bool), ob)
+
+
+def test_map_indices_small_blocks_and_bad_entries():
+    cnt = torch.tensor([[[2, 1]]], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[[1, 7, -1], [2, -1, -1]]], dtype=torch.int32, device="cuda")
+    st = _status()
+    dc, di, _ = ops.sparvar_map_indices(cnt, idx, 4, 6, 8, 15, 2, 2, n_sink_tokens=1, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & ops.SPARVAR_DEV_BAD_LIST
+    # the golden case P of tests/golden/map_indices_tiny.txt (entry 7 is skipped)
+    want = [[0, 2, 3, 4], [0, 2, 3, 4], [0, 5, 6, 7], [0, 5, 6, 7]]
+    for qb, w in enumerate(want):
+        assert di[0, 0, qb, :dc[0, 0, qb]].tolist() == w

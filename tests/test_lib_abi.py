@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host (no GPU needed: nothing is enqueued on failure)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_cross_sparvar_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sparvar.h")).read()
+    return sorted(set(re.findall(r"SPARVAR_API\s+(?:const\s+)?\w+\*?\s+(sparvar_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(ops.EXPORTS), "binding and header disagree"
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.sparvar_version()
+
+
+def test_scale_blocks_host_only(lib):
+    assert ops.scale_blocks([1, 2, 4, 6, 8, 12, 16, 20, 24, 32, 40, 48, 64], 12, 128, 128) == (32, 83)
+    assert ops.scale_blocks([1, 2, 4, 8, 16], 4, 16, 16) == (16, 22)
+    with pytest.raises(ops.SparvarError, match="q_scale"):
+        ops.scale_blocks([1, 2], 5, 128, 128)
+
+
+def _attn_call(lib, **over):
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    args = dict(q=16, k=16, v=16, o=16, lse=0, B=1, H=1, Lq=128, Lkv=128, D=128,
+                qs=i64(0, 0, 128), ks=i64(0, 0, 128), vs=i64(0, 0, 128), os=i64(0, 0, 128),
+                cnt=16, idx=16, ls=i64(0, 0), row=1, bq=128, bk=128, scale=0.1, st=0, stream=0)
+    args.update(over)
+    vp = ctypes.c_void_p
+    return lib.sparvar_block_sparse_attn_fwd(
+        vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["o"]), vp(args["lse"]), args["B"],
+        args["H"], args["Lq"], args["Lkv"], args["D"], args["qs"], args["ks"], args["vs"], args["os"],
+        vp(args["cnt"]), vp(args["idx"]), args["ls"], args["row"], args["bq"], args["bk"],
+        args["scale"], vp(args["st"]), vp(args["stream"]))
+
+
+@pytest.mark.parametrize("over,code,msg", [
+    (dict(D=96), 2, "D=96"),
+    (dict(bq=64), 2, "128 x 128"),
+    (dict(q=0), 1, "q is NULL"),
+    (dict(k=8), 1, "not 16-byte aligned"),
+    (dict(Lq=0), 1, "Lq=0"),
+    (dict(cnt=0), 1, "kv_cnt"),
+    (dict(row=-1), 1, "idx_row_len"),
+    (dict(scale=float("inf")), 1, "softmax_scale"),
+])
+def test_attention_rejects_bad_arguments_on_host(lib, over, code, msg):
+    assert _attn_call(lib, **over) == code
+    assert msg in lib.sparvar_last_error().decode()
+
+
+def test_attention_rejects_bad_strides(lib):
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    assert _attn_call(lib, qs=i64(0, 0, 100)) == 1
+    assert "row stride" in lib.sparvar_last_error().decode()
+    assert _attn_call(lib, H=2, ks=i64(0, 0, 128)) == 1
+    assert "head stride" in lib.sparvar_last_error().decode()
+
+
+def test_csla_rejects_bad_arguments(lib):
+    sides = (ctypes.c_int32 * 3)(1, 2, 4)
+    vp = ctypes.c_void_p
+    assert lib.sparvar_build_csla_mask(sides, 3, 2, 1, 0, 0, 48, 128, vp(16), vp(16), vp(0), vp(0)) == 2
+    assert lib.sparvar_build_csla_mask(sides, 3, 3, 1, 0, 0, 128, 128, vp(16), vp(16), vp(0), vp(0)) == 1
+    assert lib.sparvar_build_csla_mask(sides, 3, 2, 1, -1, 0, 128, 128, vp(16), vp(16), vp(0), vp(0)) == 1
+    bad = (ctypes.c_int32 * 3)(1, 0, 4)
+    assert lib.sparvar_build_csla_mask(bad, 3, 2, 1, 0, 0, 128, 128, vp(16), vp(16), vp(0), vp(0)) == 1
+    assert "sides[1]" in lib.sparvar_last_error().decode()
+
+
+def test_map_and_decide_reject_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    assert lib.sparvar_map_indices(vp(16), vp(16), 1, 1, 10, 10, 20, 20, 100, 128, 0, vp(16), vp(16),
+                                   vp(0), vp(0), vp(0)) == 2
+    assert lib.sparvar_map_indices(vp(0), vp(16), 1, 1, 10, 10, 20, 20, 128, 128, 0, vp(16), vp(16),
+                                   vp(0), vp(0), vp(0)) == 1
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    assert lib.sparvar_decide_blocks(vp(16), vp(16), 1, 1, 128, 600000, 128, i64(0, 0, 128),
+                                     i64(0, 0, 128), 0.1, vp(0), 128, 128, 0.95, vp(16), vp(16),
+                                     vp(0), vp(0), vp(0)) == 2
+    assert "KV blocks" in lib.sparvar_last_error().decode()
+    assert lib.sparvar_validate_lists(vp(16), vp(16), 4, 4, 4, vp(0), vp(0)) == 1
