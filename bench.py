@@ -54,13 +54,13 @@ def kept_flops_from_lists(cnt, idx, nq, L, bq, bk, D):
 
 
 def start_clock_sampler(path):
-    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     try:
         f = open(path, "w")
         return subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                 "-lms", "100"], stdout=f, stderr=subprocess.DEVNULL), f
+                                 "-lms", "20"], stdout=f, stderr=subprocess.DEVNULL), f
     except Exception:
         return None, None
 
@@ -77,7 +77,7 @@ def stop_clock_sampler(proc, f, path, gpu_index):
     sm, mx, reasons = [], 0.0, set()
     names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     for line in open(path):
-        parts = [p.strip() for p in line.split(",")]
+        parts = [p.strip() for p in line.split(",")][1:]
         if len(parts) < 9 or parts[0] != str(gpu_index):
             continue
         try:
@@ -91,42 +91,50 @@ def stop_clock_sampler(proc, f, path, gpu_index):
     if not sm:
         return None
     return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "samples": len(sm),
-            "reasons": sorted(reasons)}
+            "reasons": sorted(reasons), "window": "1 s of back-to-back steps + the timed region"}
 
 
-def cpu_baseline(wl, budget_s=12.0, seed=0):
+def cpu_baseline(wl, budget_s=12.0, seed=0, d=None):
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
-    one (batch, head) and as many query blocks as fit in ``budget_s``."""
+    (batch, head) pairs one after another, query block by query block, until
+    ``budget_s`` of CPU time has been spent."""
     from oracle import sparvar_oracle as orc
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         threads = len(os.sched_getaffinity(0))
-    sides, k = wl["sides"], wl["q_scale"]
-    d = inputs.make_qkv(seed, 1, 1, sides, wl["D"], wl["n_sink_scales"])
+    sides, k, bq = wl["sides"], wl["q_scale"], wl["block"]
+    if d is None:
+        d = inputs.make_qkv(seed, wl["B"], wl["H"], sides, wl["D"], wl["n_sink_scales"])
     off = d["offsets"]
-    f64 = lambda a: a.astype(np.float64)  # noqa: E731
-    q = f64(d["qf"][0, 0, off[k]:off[k + 1]])
-    kk = f64(d["kf"][0, 0, :off[k + 1]])
-    vv = f64(d["vf"][0, 0, :off[k + 1]])
-    bq = wl["block"]
     t0 = time.perf_counter()
-    cnt, idx, blk = orc.build_csla_mask(sides, k, wl["n_sink_scales"], wl["radius_prev"],
-                                        wl["radius_own"], bq, bq)
-    nq, L = q.shape[0], kk.shape[0]
-    flops, done = 0, 0
-    while done < blk.shape[0] and time.perf_counter() - t0 < budget_s:
-        rows = np.arange(done * bq, min((done + 1) * bq, nq))
-        orc.masked_attention_rows(rows, q, kk, vv, blk, bq, bq)
-        sub = np.zeros_like(blk)
-        sub[done] = blk[done]
-        flops += orc.kept_flops(sub, nq, L, bq, bq, wl["D"])
-        done += 1
+    flops, blocks, pairs = 0, 0, 0
+    for b in range(wl["B"]):
+        for h in range(wl["H"]):
+            if time.perf_counter() - t0 >= budget_s:
+                break
+            q = d["qf"][b, h, off[k]:off[k + 1]].astype(np.float64)
+            kk = d["kf"][b, h, :off[k + 1]].astype(np.float64)
+            vv = d["vf"][b, h, :off[k + 1]].astype(np.float64)
+            cnt, idx, blk = orc.build_csla_mask(sides, k, wl["n_sink_scales"], wl["radius_prev"],
+                                                wl["radius_own"], bq, bq)
+            nq, L = q.shape[0], kk.shape[0]
+            pairs += 1
+            for qb in range(blk.shape[0]):
+                if time.perf_counter() - t0 >= budget_s:
+                    break
+                rows = np.arange(qb * bq, min((qb + 1) * bq, nq))
+                orc.masked_attention_rows(rows, q, kk, vv, blk, bq, bq)
+                sub = np.zeros_like(blk)
+                sub[qb] = blk[qb]
+                flops += orc.kept_flops(sub, nq, L, bq, bq, wl["D"])
+                blocks += 1
     dt = time.perf_counter() - t0
+    nqb = -(-(off[k + 1] - off[k]) // bq)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
-            "sample": f"1 of {wl['B'] * wl['H']} (batch, head) pairs, {done} of {blk.shape[0]} query "
-                      f"blocks, CSLA mask build included; numpy fp64 ({dt:.1f} s)",
+            "sample": f"{blocks} of {wl['B'] * wl['H'] * nqb} (batch, head, query block) units over "
+                      f"{pairs} (batch, head) pairs, CSLA mask build included; numpy fp64, {dt:.1f} s",
             "seconds": dt}
 
 
@@ -134,9 +142,10 @@ def run_reference(args, wl, rank, world):
     if world > 1 and rank != 0:
         return
     per_step = []
-    res = None
+    d = inputs.make_qkv(0, wl["B"], wl["H"], wl["sides"], wl["D"], wl["n_sink_scales"])
+    budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        res = cpu_baseline(wl, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)), seed=0)
+        res = cpu_baseline(wl, budget_s=budget, d=d)
         if i >= args.warmup:
             per_step.append(res)
     val = float(np.mean([r["value"] for r in per_step]))
@@ -161,6 +170,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="seconds of untimed back-to-back steps while the clock sampler starts")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -219,7 +230,12 @@ def main():
     clocks_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") \
         if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/sparvar_clocks_{rank}.csv"
     sampler, sf = start_clock_sampler(clocks_path) if rank == 0 else (None, None)
-    time.sleep(0.3 if sampler else 0)
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak_s:  # same load as the timed steps, untimed
+        for _ in range(20):
+            flush.fill_(0)
+            step(q, kk, vv, o)
+        torch.cuda.synchronize()
 
     if world > 1:
         dist.barrier()

@@ -311,13 +311,15 @@ def test_map_indices_bit_exact(dst_scale):
 
 
 def test_map_indices_small_blocks_and_bad_entries():
+    # golden case P of tests/golden/map_indices_tiny.txt with every size times 16
+    # (block 32 instead of 2): the same destination blocks must come out.
     cnt = torch.tensor([[[2, 1]]], dtype=torch.int32, device="cuda")
-    idx = torch.tensor([[[1, 7, -1], [2, -1, -1]]], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[[[1, 7, -1], [2, -1, -1]]]], dtype=torch.int32, device="cuda")
     st = _status()
-    dc, di, _ = ops.sparvar_map_indices(cnt, idx, 4, 6, 8, 15, 2, 2, n_sink_tokens=1, dev_status=st)
+    dc, di, _ = ops.sparvar_map_indices(cnt, idx, 64, 96, 128, 240, 32, 32, n_sink_tokens=16,
+                                        dev_status=st)
     torch.cuda.synchronize()
-    assert st.item() & ops.SPARVAR_DEV_BAD_LIST
-    # the golden case P of tests/golden/map_indices_tiny.txt (entry 7 is skipped)
+    assert st.item() & ops.SPARVAR_DEV_BAD_LIST  # entry 7 is out of range and skipped
     want = [[0, 2, 3, 4], [0, 2, 3, 4], [0, 5, 6, 7], [0, 5, 6, 7]]
     for qb, w in enumerate(want):
         assert di[0, 0, qb, :dc[0, 0, qb]].tolist() == w
