@@ -281,11 +281,9 @@ def main():
     t_step = float(np.mean(step_ms))
     t_attn = float(np.mean(attn_ms))
     t_e2e = float(np.mean(e2e_ms))
-    if world > 1:
-        tt = torch.tensor([t_step, t_attn, t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_attn, t_e2e = tt.tolist()
-    total_flops = flops_step * world
+    from block_sparse_cross_sparvar_b200 import multi
+    t_step, t_attn, t_e2e = multi.max_over_ranks([t_step, t_attn, t_e2e], dev)
+    (total_flops,) = multi.sum_over_ranks([float(flops_step)], dev)
     pk = peaks()
     if rank == 0:
         achieved = flops_step / (t_attn * 1e-3) / 1e12

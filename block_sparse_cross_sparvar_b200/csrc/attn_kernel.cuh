@@ -24,6 +24,7 @@
 #include <cuda.h>
 
 #include "ptx.cuh"
+#include "tmem_io.cuh"
 
 namespace sparvar {
 
@@ -106,7 +107,7 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
+                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs args) {
   using L = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
@@ -310,8 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          tmem_ld32(s_addr + cc * 32, r);
-          tmem_wait_ld();
+          tmem_ld32_wait(s_addr + cc * 32, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]) * c;
         }
@@ -358,8 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t r[32];
-            tmem_ld32(o_addr + cc * 32, r);
-            tmem_wait_ld();
+            tmem_ld32_wait(o_addr + cc * 32, r);
 #pragma unroll
             for (int i2 = 0; i2 < 32; ++i2) r[i2] = __float_as_uint(__uint_as_float(r[i2]) * alpha);
             tmem_st32(o_addr + cc * 32, r);
@@ -426,8 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
           if (n_blocks > 0) {
-            tmem_ld32(o_addr + cc * 32, r);
-            tmem_wait_ld();
+            tmem_ld32_wait(o_addr + cc * 32, r);
           } else {
 #pragma unroll
             for (int i2 = 0; i2 < 32; ++i2) r[i2] = 0u;

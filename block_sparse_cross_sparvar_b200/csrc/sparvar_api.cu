@@ -11,6 +11,7 @@
 #include <string>
 
 #include "../../include/sparvar.h"
+#include "attn_fwd_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "mask_kernels.cuh"
 
@@ -127,6 +128,21 @@ int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   kern<<<grid, sparvar::kThreads, smem, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "block_sparse_attn_kernel launch");
+  return SPARVAR_OK;
+}
+
+template <int D>
+int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const sparvar::fwd::Args& a, cudaStream_t stream) {
+  auto kern = sparvar::fwd::attn_fwd_kernel<D>;
+  const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  dim3 grid(a.nqb, a.H, a.B);
+  kern<<<grid, sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return SPARVAR_OK;
 }
 
@@ -258,9 +274,10 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   if (list_strides[0] < 0 || list_strides[1] < 0)
     return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
   if (idx_row_len < 0) return fail(SPARVAR_ERR_INVALID_ARG, "idx_row_len < 0");
-  if (!std::isfinite(softmax_scale)) return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale not finite");
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f))
+    return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
 
-  sparvar::AttnArgs a{};
+  sparvar::fwd::Args a{};
   a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
   a.nqb = static_cast<int>(ceil_div(Lq, 128));
   a.nkb = static_cast<int>(ceil_div(Lkv, 128));
@@ -270,7 +287,7 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   a.idx_row_len = idx_row_len;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
-  a.lse_out = lse;
+  a.lse = lse;
   a.dev_status = dev_status;
 
   CUtensorMap tq, tk, tv;
@@ -278,8 +295,8 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
   if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_attn_kernel<128, sparvar::kModeAttn>(tq, tk, tv, a, st);
-  return launch_attn_kernel<64, sparvar::kModeAttn>(tq, tk, tv, a, st);
+  if (D == 128) return launch_fwd_kernel<128>(tq, tk, tv, a, st);
+  return launch_fwd_kernel<64>(tq, tk, tv, a, st);
 }
 
 int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
@@ -303,8 +320,8 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   if ((rc = check_operand(q, q_strides, B, H, Lq, D, "q"))) return rc;
   if ((rc = check_operand(k, k_strides, B, H, Lkv, D, "k"))) return rc;
   if (!kv_cnt || !kv_idx) return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx is NULL");
-  if (!std::isfinite(softmax_scale) || std::isnan(mass_threshold))
-    return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale or mass_threshold not a number");
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f) || std::isnan(mass_threshold))
+    return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0, mass_threshold a number");
 
   sparvar::AttnArgs a{};
   a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
