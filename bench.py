@@ -170,6 +170,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", action="store_true",
+                    help="after the main line, print one line per further workload (CS4A full pass, "
+                         "Infinity-8B radius sweep, density sweep)")
     ap.add_argument("--soak-s", type=float, default=1.0,
                     help="seconds of untimed back-to-back steps while the clock sampler starts")
     args = ap.parse_args()
@@ -318,6 +321,13 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = {kk_: v for kk_, v in cpu_baseline(wl).items() if kk_ != "seconds"}
         print(json.dumps(line), flush=True)
+        if args.extra and world == 1:
+            from block_sparse_cross_sparvar_b200 import workloads
+            del q, kk, vv, o, hq, hk, hv
+            torch.cuda.empty_cache()
+            for fn in (workloads.cs4a_full_pass, workloads.csla_radius_sweep, workloads.density_sweep):
+                print(json.dumps({"extra": fn(dev)}), flush=True)
+                torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
 

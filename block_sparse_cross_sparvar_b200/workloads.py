@@ -1,0 +1,176 @@
+"""GPU runs of the Infinity-shaped workloads beyond the headline last scale.
+
+* ``cs4a_full_pass``: all 13 scales of one generation step with CS4A: scales
+  1-10 dense (the 32x32 scale also yields the row LSE), the decision on the
+  32x32 scale (pooled mass >= 0.95), and the mapped lists for 40x40, 48x48 and
+  64x64.
+* ``csla_radius_sweep``: the Infinity-8B-like last two scales (B2 H32) with the
+  CSLA locality radius of earlier scales at 1, 2 and 4.
+* ``density_sweep``: the last scale with random block lists at fixed densities
+  (sink block always kept), with the full key prefix and with the 40x40 and
+  48x48 scales skipped from the prefix.
+
+Every step runs in the library's kernels; torch only provides memory, streams
+and events.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import inputs, ops
+
+FLUSH_BYTES = 256 << 20
+
+
+def _dev(bits, device):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def _dense_lists(nqb, nkb, device):
+    cnt = torch.full((nqb,), nkb, dtype=torch.int32, device=device)
+    idx = torch.arange(nkb, dtype=torch.int32, device=device).repeat(nqb, 1).contiguous()
+    return cnt, idx
+
+
+def kept_flops(cnt, idx, nq, L, block, D):
+    """4 * n_q * n_k * D over kept blocks (host copy of the lists)."""
+    cnt = cnt.cpu().numpy()
+    idx = idx.cpu().numpy()
+    lead = cnt.shape[:-1]
+    cnt2 = cnt.reshape(-1, cnt.shape[-1])
+    idx2 = idx.reshape(-1, idx.shape[-2], idx.shape[-1])
+    total = 0
+    for r in range(cnt2.shape[0]):
+        for qb in range(cnt2.shape[1]):
+            nqr = min((qb + 1) * block, nq) - qb * block
+            for kb in idx2[r, qb, :cnt2[r, qb]]:
+                total += 4 * nqr * (min((int(kb) + 1) * block, L) - int(kb) * block) * D
+    return total, int(np.prod(lead)) if lead else 1
+
+
+def time_ms(fn, reps, device, warmup=3):
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    out = []
+    for i in range(reps):
+        flush.fill_(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        out.append(a.elapsed_time(b))
+    return float(np.median(out))
+
+
+def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision_scale=9):
+    sides = inputs.INFINITY_SIDES
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    q_all, k_all, v_all = _dev(d["q"], device), _dev(d["k"], device), _dev(d["v"], device)
+    del d
+    n_scales = len(sides)
+    outs = [torch.empty(B, H, off[s + 1] - off[s], D, dtype=torch.bfloat16, device=device)
+            for s in range(n_scales)]
+    dense = [_dense_lists(-(-(off[s + 1] - off[s]) // 128), -(-off[s + 1] // 128), device)
+             for s in range(decision_scale + 1)]
+    state = {}
+
+    def run():
+        for s in range(decision_scale + 1):
+            q = q_all[:, :, off[s]:off[s + 1]]
+            k = k_all[:, :, :off[s + 1]]
+            v = v_all[:, :, :off[s + 1]]
+            cnt, idx = dense[s]
+            if s == decision_scale:
+                _, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=outs[s], return_lse=True)
+                dc, di, _ = ops.sparvar_decide_blocks(q, k, tau, lse=lse)
+                state["dec"] = (dc, di)
+            else:
+                ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=outs[s])
+        dc, di = state["dec"]
+        src_nq, src_lkv = off[decision_scale + 1] - off[decision_scale], off[decision_scale + 1]
+        for s in range(decision_scale + 1, n_scales):
+            nq, L = off[s + 1] - off[s], off[s + 1]
+            mc, mi, _ = ops.sparvar_map_indices(dc, di, src_nq, src_lkv, nq, L, 128, 128, off[5])
+            state[s] = (mc, mi)
+            ops.sparvar_block_sparse_attn_fwd(q_all[:, :, off[s]:off[s + 1]], k_all[:, :, :L],
+                                              v_all[:, :, :L], mc, mi, out=outs[s])
+
+    ms = time_ms(run, reps, device)
+    flops = 0
+    per_scale = {}
+    for s in range(n_scales):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        if s <= decision_scale:
+            f = 4 * nq * L * D * B * H
+        else:
+            f, _ = kept_flops(*state[s], nq, L, 128, D)
+        per_scale[f"{sides[s]}x{sides[s]}"] = {"gflop": f / 1e9,
+                                                "density": f / (4 * nq * L * D * B * H)}
+        flops += f
+    return {"workload": "cs4a_full_pass_13_scales", "B": B, "H": H, "D": D, "tau": tau,
+            "ms": ms, "gflop": flops / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
+            "scales": per_scale}
+
+
+def csla_radius_sweep(device, reps=10, seed=0, B=2, H=32, D=128, radii=(1, 2, 4)):
+    sides = inputs.INFINITY_SIDES
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    q_all, k_all, v_all = _dev(d["q"], device), _dev(d["k"], device), _dev(d["v"], device)
+    del d
+    res = []
+    for s in (11, 12):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        q = q_all[:, :, off[s]:off[s + 1]]
+        out = torch.empty_like(q)
+        for r in radii:
+            cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, 5, r, 4, 128, 128, device=device)
+            ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k_all[:, :, :L], v_all[:, :, :L],
+                                                                   cnt, idx, out=out), reps, device)
+            f, _ = kept_flops(cnt, idx, nq, L, 128, D)
+            f *= B * H
+            res.append({"scale": f"{sides[s]}x{sides[s]}", "radius_prev": r, "radius_own": 4,
+                        "density": f / (4 * nq * L * D * B * H), "ms": ms,
+                        "tflops": f / (ms * 1e-3) / 1e12})
+    return {"workload": "infinity8b_last_two_scales_csla_radius_sweep", "B": B, "H": H, "D": D,
+            "runs": res}
+
+
+def density_sweep(device, reps=10, seed=0, B=2, H=16, D=128, densities=(0.05, 0.1, 0.2, 0.35, 0.5, 1.0)):
+    sides = inputs.INFINITY_SIDES
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    rng = d["rng"]
+    q = _dev(d["q"][:, :, off[12]:off[13]], device)
+    prefixes = {"full_10521": np.arange(off[13]),
+                "skip_40_48_6617": np.concatenate([np.arange(off[10]), np.arange(off[12], off[13])]),
+                "skip_7225": np.arange(7225)}
+    res = []
+    for name, keys in prefixes.items():
+        k = _dev(np.ascontiguousarray(d["k"][:, :, keys]), device)
+        v = _dev(np.ascontiguousarray(d["v"][:, :, keys]), device)
+        L = keys.size
+        nqb, nkb = 32, -(-L // 128)
+        out = torch.empty_like(q)
+        for dens in densities:
+            keep = inputs.bernoulli_keep(rng, (B, H, nqb, nkb), dens)
+            keep[..., 0] = True
+            cnt = torch.from_numpy(keep.sum(-1).astype(np.int32)).to(device)
+            idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
+            for bb in range(B):
+                for hh in range(H):
+                    for qb in range(nqb):
+                        kept = np.nonzero(keep[bb, hh, qb])[0]
+                        idx_np[bb, hh, qb, :kept.size] = kept
+            idx = torch.from_numpy(idx_np).to(device)
+            ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=out), reps, device)
+            f, _ = kept_flops(cnt, idx, 4096, L, 128, D)
+            res.append({"prefix": name, "Lkv": L, "target_density": dens,
+                        "density": f / (4 * 4096 * L * D * B * H), "ms": ms,
+                        "tflops": f / (ms * 1e-3) / 1e12})
+    return {"workload": "last_scale_density_sweep", "B": B, "H": H, "D": D, "runs": res}
