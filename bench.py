@@ -43,6 +43,25 @@ def peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
+def profiled_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    import hashlib
+    try:
+        src = os.path.join(ROOT, "block_sparse_cross_sparvar_b200", "csrc", "attn_fwd_kernel.cuh")
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        fields = {}
+        for line in open(os.path.join(ROOT, "profiles", "attn_fwd_infinity2b_last.md")):
+            if ":" in line and not line.startswith("|"):
+                key, _, val = line.partition(":")
+                fields[key.strip()] = val.strip()
+        if fields.get("kernel_source_sha256_16") == sha:
+            return int(fields["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
 def kept_flops_from_lists(cnt, idx, nq, L, bq, bk, D):
     total = 0
     for qb in range(cnt.shape[0]):
@@ -306,11 +325,13 @@ def main():
                        "kept_gflop_per_step_per_gpu": flops_step / 1e9,
                        "l2": "256 MB flush write between timed steps",
                        "parallelism": f"independent batch per GPU x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "block_sparse_attn_kernel<128,0>",
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
                          "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16"],
                          "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']}",
-                         "traffic": None},
+                         "traffic": profiled_traffic(),
+                         "traffic_note": "ncu dram bytes read+write per launch (profiles/attn_fwd_infinity2b_last.md); "
+                                         "null when the kernel source changed since"},
             "e2e": {"value": total_flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": t_e2e,
                     "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),

@@ -1,33 +1,45 @@
-// Block-sparse attention forward on sm_100a.
+// Block-sparse attention forward on sm_100a: a persistent kernel.
 //
-// One CTA owns one 128-row query tile (one query block of one batch item and
-// head) and walks that tile's list of KV blocks j = 0 .. n-1.  Roles:
-//   warps 0-3   softmax group 0: blocks j = 0, 2, 4, ... (thread t: query row t,
+// Each CTA owns one SM and walks the query tiles t = blockIdx.x, blockIdx.x +
+// gridDim.x, ... (a tile is one 128-row query block of one batch item and
+// head).  The KV blocks of all its tiles form one block sequence J = 0, 1, ...
+// (tile after tile), and the pipeline runs across tile boundaries: the next
+// tile's Q, first K blocks and first score MMAs overlap the current tile's last
+// blocks and its epilogue.  Roles:
+//   warps 0-3   softmax group 0: blocks with J even (thread t: query row t,
 //               TMEM lane t)
-//   warps 4-7   softmax group 1: blocks j = 1, 3, 5, ...
-//   warp  8     MMA issue for even blocks (one lane) and TMEM owner
+//   warps 4-7   softmax group 1: blocks with J odd
+//   warp  8     MMA issue for even J (one lane), tile prologues, TMEM owner
 //   warp  9     TMA producer (one lane)
-//   warp  10    MMA issue for odd blocks (one lane)
-// TMEM (512 columns): three score buffers S_b = [128b, 128b+128), b = j mod 3,
-// and the output accumulator O = [384, 384+D).  P_j is written as packed bf16
+//   warp  10    MMA issue for odd J (one lane)
+// TMEM (512 columns): three score buffers S_b = [128b, 128b+128), b = J mod 3,
+// and the output accumulator O = [384, 384+D).  P_J is written as packed bf16
 // over the first 64 columns of its score buffer and feeds the PV MMA from TMEM.
-// The MMA warp keeps three score blocks in flight (S_{j+3} is issued right
-// after PV_j, which frees buffer j mod 3), so a softmax group finds its next S
-// already computed and the tensor core never waits for a softmax round trip.
-// Q is loaded once; K and V blocks pass through a ring of shared-memory slots
-// in the order the MMA warp needs them: K_0, K_1, K_2, then V_j, K_{j+3}.  The
-// MMA warp issues PV_j and S_{j+3} as one group and frees both slots with one
-// commit.
+// Shared memory: two Q buffers (the k-th non-empty tile uses Q[k mod 2]) and a
+// ring of K/V slots.  Within a tile of n blocks the ring order is K_0..K_{n0-1}
+// (n0 = min(n, 3)), then V_j and, while j + 3 < n, K_{j+3}.
 //
-// Both groups add into the one O accumulator, so they share a per-row
-// reference max m (log2 units) in shared memory.  Block j is computed against
-// the reference read when it starts and finalised in block order: its group
-// waits until block j-1 has been handed to the MMA warp, re-reads m, and either
-// raises m (when the block's max exceeds m by more than 2^8: O is rescaled in
-// place once PV_{j-1} has completed, i.e. once group j-1 has released its slots)
-// or, if m moved meanwhile, rescales its own
-// P in TMEM.  Each group keeps its row sum relative to its own last reference;
-// the epilogue combines the two sums against the final m.
+// MMA groups.  A tile's prologue (S_0 .. S_{n0-1}) is one group, issued by
+// issuer 0 once the previous tile's MMAs have all completed.  Block j's group
+// is PV_j followed by S_{j+3} into the buffer PV_j has just read (one issuer's
+// MMAs run in issue order); issuer J mod 2 runs it, so while one issuer waits
+// on a barrier the other keeps the tensor core's short queue filled.  Each
+// group commits once on rel[G mod 16] (G numbers the groups of the sequence in
+// order), which frees its ring slots; the producer records, per slot, the group
+// that must release it.  Release barriers outnumber ring slots, so no waiter can
+// fall two phases behind a barrier.
+//
+// Softmax.  Both groups add into one O, so they share a per-row reference max
+// m (log2 units) in shared memory, reset at each tile.  Block J is computed
+// against the reference read when it starts and finalised in block order: its
+// group waits until P_{J-1} has been handed over, re-reads m, and either raises
+// m (block max more than 2^8 above it: O is rescaled in place once the tile's
+// earlier PVs have completed) or, if m moved meanwhile, rescales its own P in
+// TMEM.  O is zeroed before a tile's first PV, so the two issuers' PVs may
+// accumulate in either order.  The epilogue waits for the tile's last two
+// groups, merges the two groups' row sums against the final m (exchanging them
+// through the tile's Q buffer, which no MMA reads any more), writes O and the
+// LSE, and hands the Q buffer back to the producer.
 #pragma once
 
 #include <cuda.h>
@@ -41,14 +53,19 @@ namespace fwd {
 
 constexpr int kTile = 128;
 constexpr int kThreads = 352;
-constexpr int kMmaWarp = 8;    // MMA issuer 0 (even blocks) and TMEM owner
+constexpr int kMmaWarp = 8;    // MMA issuer 0 (even J), tile prologues, TMEM owner
 constexpr int kLoadWarp = 9;
-constexpr int kMmaWarp1 = 10;  // MMA issuer 1 (odd blocks), on another SM sub-partition
+constexpr int kMmaWarp1 = 10;  // MMA issuer 1 (odd J), on another SM sub-partition
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 384;
 constexpr float kLazyRescale = 8.0f;          // log2 units
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
 constexpr uint64_t kDrainNs = 500000000ull;   // 0.5 s per drain
 constexpr int kMaxSlots = 12;
+constexpr int kRel = 16;                      // release barriers (more than ring slots)
+// Of each 16 pairs of score columns, those whose bit is set take the FMA-pipe 2^x
+// (exp2_poly2), the others the MUFU ex2.
+constexpr uint32_t kPolyPairs = 0x0u;
 
 struct Args {
   int B, H, Lq, Lkv, nqb, nkb;
@@ -64,49 +81,85 @@ struct Args {
 };
 
 struct __align__(8) Bars {
-  uint64_t q_full;
+  uint64_t q_full[2];             // Q of non-empty tile k landed: [k & 1], phase k >> 1
+  uint64_t epi[2];                // epilogue of non-empty tile k done: [k & 1], phase k >> 1
   uint64_t full[kMaxSlots];       // ring slot loaded (TMA transaction count)
-  uint64_t rel[8];                // group j (PV_j and S_{j+3}) done: its ring slots are free
-  uint64_t pro_done;              // prologue score groups done: K_0..K_2 slots are free
-  uint64_t s_full[3], p_full[3];  // per score buffer
-  uint64_t o_done;
+  uint64_t rel[kRel];             // MMA group G done: [G % kRel], phase G / kRel
+  uint64_t s_full[3], p_full[3];  // block J: [J % 3], phase J / 3
   uint64_t drain;
 };
-
-// Ring positions: K_0 .. K_{n0-1} (n0 = min(n, 3)), then V_j and, while j + 3 < n,
-// K_{j+3}, for j = 0 .. n-1.  The group that consumes position p (or the prologue)
-// is what frees its slot.  Group j commits on rel[j % 8]: a slot is reused five
-// positions later, so its user is at most ~3 groups ahead of the group that
-// freed it and a waiter can never be two phases behind on that barrier.
-__device__ __forceinline__ int ring_pos_v(int j, int n) {
-  const int n0 = n < 3 ? n : 3;
-  const int nk = n > 3 ? n - 3 : 0;
-  return n0 + j + (j < nk ? j : nk);
-}
-// block whose group consumes ring position p >= n0
-__device__ __forceinline__ int ring_block(int p, int n) {
-  const int n0 = n < 3 ? n : 3;
-  const int nk = n > 3 ? n - 3 : 0;
-  const int q = p - n0;
-  return q < 2 * nk ? (q >> 1) : nk + (q - 2 * nk);
-}
 
 template <int D>
 struct Layout {
   static constexpr uint32_t kTileBytes = kTile * D * 2;
   static constexpr uint32_t kChunkBytes = kTile * 128;  // 128 rows x 64 bf16
   static constexpr int kChunks = D / 64;
-  static constexpr int kSlots = D == 128 ? 6 : 12;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kRing = kTileBytes;
-  static constexpr uint32_t kColO = 384;
-  static constexpr uint32_t kBytes = (1 + kSlots) * kTileBytes + 1024;
+  static constexpr int kSlots = D == 128 ? 5 : 12;
+  static constexpr uint32_t kQ = 0;  // two Q buffers
+  static constexpr uint32_t kRing = 2 * kTileBytes;
+  static constexpr uint32_t kBytes = (2 + kSlots) * kTileBytes + 1024;
 };
+
+// One tile of this CTA's sequence, with the sequence counters at its start.
+struct TileCursor {
+  int t;  // tile id (b * H + h) * nqb + qb; >= total when the CTA is done
+  int n;  // list length (clamped to [0, idx_row_len])
+  const int32_t* list;
+  int J0;    // sequence index of the tile's first block
+  int pos0;  // ring position of the tile's first operand
+  int k;     // number of non-empty tiles before this one
+};
+
+struct TileCoord {
+  int b, h, qb;
+};
+__device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
+  const int bh = t / a.nqb;
+  return TileCoord{bh / a.H, bh % a.H, t % a.nqb};
+}
+
+__device__ __forceinline__ void cursor_load(TileCursor& c, const Args& a, int total, bool report) {
+  if (c.t >= total) return;
+  const TileCoord tc = tile_coord(c.t, a);
+  const int64_t lrow = tc.b * a.list_sb + tc.h * a.list_sh + tc.qb;
+  int n = __ldg(a.kv_cnt + lrow);
+  if (n < 0 || n > a.idx_row_len) {
+    if (report && a.dev_status) atomicOr(a.dev_status, 0x1);
+    n = n < 0 ? 0 : a.idx_row_len;
+  }
+  c.n = n;
+  c.list = a.kv_idx + lrow * a.idx_row_len;
+}
+
+__device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int total, bool report) {
+  if (c.n > 0) {
+    const int n0 = c.n < 3 ? c.n : 3;
+    const int nk = c.n > 3 ? c.n - 3 : 0;
+    c.J0 += c.n;
+    c.pos0 += n0 + c.n + nk;
+    c.k += 1;
+  }
+  c.t += gridDim.x;
+  cursor_load(c, a, total, report);
+}
+
+__device__ __forceinline__ int group_of_prologue(const TileCursor& c) { return c.J0 + c.k; }
+__device__ __forceinline__ int group_of_block(const TileCursor& c, int j) {
+  return c.J0 + c.k + 1 + j;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* st) {
   const bool ok = mbar_wait(bar, parity, abort, st, 0x2, kWaitNs);
   return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool wait_group(uint64_t* rel, int grp, volatile int* abort,
+                                           int32_t* st) {
+  return mbar_wait(&rel[grp % kRel], (grp / kRel) & 1, abort, st, 0x2, kWaitNs);
+}
+__device__ __forceinline__ bool warp_wait_group(uint64_t* rel, int grp, volatile int* abort,
+                                                int32_t* st) {
+  return warp_wait(&rel[grp % kRel], (grp / kRel) & 1, abort, st);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -126,38 +179,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Bars bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float m_sh[kTile];  // shared reference max per row
+  __shared__ float m_sh[kTile];      // shared reference max per row
+  __shared__ int relg_sh[kMaxSlots];  // producer: group that frees each ring slot (-1: unused)
 
   const uint32_t smem_base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_addr(smem_raw));
   const int warp = warp_id();
   const int lane = lane_id();
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   volatile int* abort_flag = &abort_sh;
   int32_t* dev_status = args.dev_status;
-
-  const int64_t lrow = b * args.list_sb + h * args.list_sh + qb;
-  int n = __ldg(args.kv_cnt + lrow);
-  if (n < 0 || n > args.idx_row_len) {
-    if (threadIdx.x == 0 && dev_status) atomicOr(dev_status, 0x1);
-    n = n < 0 ? 0 : args.idx_row_len;
-  }
-  const int32_t* list = args.kv_idx + lrow * args.idx_row_len;
+  const int total = args.B * args.H * args.nqb;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
-    mbar_init(&bars.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.epi[i], 1);
+    }
+    for (int s = 0; s < NS; ++s) mbar_init(&bars.full[s], 1);
+    for (int i = 0; i < kRel; ++i) mbar_init(&bars.rel[i], 1);
     for (int i = 0; i < 3; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 128);
     }
-    mbar_init(&bars.o_done, 2);  // one commit per issuer
-    for (int s = 0; s < NS; ++s) mbar_init(&bars.full[s], 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&bars.rel[i], 1);
-    mbar_init(&bars.pro_done, 1);
     mbar_init(&bars.drain, 2);  // one commit per issuer
     fence_barrier_init();
   }
   if (threadIdx.x < kTile) m_sh[threadIdx.x] = -INFINITY;
+  if (threadIdx.x < kMaxSlots) relg_sh[threadIdx.x] = -1;
   if (warp == kMmaWarp) {
     tmem_alloc(&tmem_base_sh, kTmemCols);
     tmem_relinquish();
@@ -171,50 +220,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t sQ = smem_base + L::kQ;
+  auto sQ = [&](int k) { return smem_base + L::kQ + (k & 1) * L::kTileBytes; };
   auto sSlot = [&](int s) { return smem_base + L::kRing + s * L::kTileBytes; };
+
+  TileCursor first{};
+  first.t = blockIdx.x;
+  cursor_load(first, args, total, threadIdx.x == 0);
 
   if (warp == kLoadWarp) {
     // ================================================================ producer
-    if (lane == 0 && n > 0) {
-      const int n0 = n < 3 ? n : 3;
+    if (lane == 0) {
       int w = 0;  // ring position
+      int q_issued0 = 0, q_issued1 = 0;  // Q loads into each buffer
       bool ok = true;
-      auto produce = [&](const CUtensorMap* tm, int kb) {
+      auto produce = [&](const CUtensorMap* tm, int kb, int grp, const TileCoord& tc) {
         const int s = w % NS;
-        if (w >= NS) {
-          // wait until the group that consumed position w - NS has completed
-          const int prev = w - NS;
-          bool got;
-          if (prev < n0) {
-            got = mbar_wait(&bars.pro_done, 0, abort_flag, dev_status, 0x2, kWaitNs);
-          } else {
-            const int jb = ring_block(prev, n);
-            got = mbar_wait(&bars.rel[jb & 7], (jb >> 3) & 1, abort_flag, dev_status, 0x2, kWaitNs);
-          }
-          if (!got) {
-            ok = false;
-            return;
-          }
+        const int prev = relg_sh[s];
+        if (prev >= 0 && !wait_group(bars.rel, prev, abort_flag, dev_status)) {
+          ok = false;
+          return;
         }
+        relg_sh[s] = grp;
         kb = kb < 0 ? -1 : (kb > args.nkb ? args.nkb : kb);
         mbar_arrive_expect_tx(&bars.full[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sSlot(s) + c * L::kChunkBytes, tm, &bars.full[s], c * 64, kb * kTile, h, b);
+          tma_load_4d(sSlot(s) + c * L::kChunkBytes, tm, &bars.full[s], c * 64, kb * kTile, tc.h,
+                      tc.b);
         ++w;
       };
-      mbar_arrive_expect_tx(&bars.q_full, L::kTileBytes);
+      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
+        if (c.n == 0) continue;
+        const int qs = c.k & 1;
+        // Q buffer qs is free once tile k - 2's epilogue is done with it
+        if (c.k >= 2 &&
+            !mbar_wait(&bars.epi[qs], ((c.k - 2) >> 1) & 1, abort_flag, dev_status, 0x2, kWaitNs)) {
+          ok = false;
+          break;
+        }
+        const TileCoord tc = tile_coord(c.t, args);
+        mbar_arrive_expect_tx(&bars.q_full[qs], L::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_4d(sQ + c * L::kChunkBytes, &tm_q, &bars.q_full, c * 64, qb * kTile, h, b);
-      for (int j = 0; j < n0 && ok; ++j) produce(&tm_k, __ldg(list + j));
-      for (int j = 0; j < n && ok; ++j) {
-        produce(&tm_v, __ldg(list + j));
-        if (ok && j + 3 < n) produce(&tm_k, __ldg(list + j + 3));
+        for (int cc = 0; cc < L::kChunks; ++cc)
+          tma_load_4d(sQ(c.k) + cc * L::kChunkBytes, &tm_q, &bars.q_full[qs], cc * 64,
+                      tc.qb * kTile, tc.h, tc.b);
+        if (qs) ++q_issued1; else ++q_issued0;
+        const int n0 = c.n < 3 ? c.n : 3;
+        for (int jj = 0; jj < n0 && ok; ++jj)
+          produce(&tm_k, __ldg(c.list + jj), group_of_prologue(c), tc);
+        for (int j = 0; j < c.n && ok; ++j) {
+          const int grp = group_of_block(c, j);
+          produce(&tm_v, __ldg(c.list + j), grp, tc);
+          if (ok && j + 3 < c.n) produce(&tm_k, __ldg(c.list + j + 3), grp, tc);
+        }
       }
       // drain: every issued TMA write lands before the CTA exits
-      mbar_drain(&bars.q_full, 0, kDrainNs);
+      if (q_issued0) mbar_drain(&bars.q_full[0], (q_issued0 - 1) & 1, kDrainNs);
+      if (q_issued1) mbar_drain(&bars.q_full[1], (q_issued1 - 1) & 1, kDrainNs);
       for (int s = 0; s < NS; ++s) {
         const int issued = w > s ? (w - 1 - s) / NS + 1 : 0;  // loads that used slot s
         if (issued) mbar_drain(&bars.full[s], (issued - 1) & 1, kDrainNs);
@@ -222,261 +284,321 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp1) {
     // ================================================================ MMA issue
-    // The tensor core queues only a few MMAs ahead of the one it executes, so
-    // a single issuing thread loses tensor time whenever it waits on a barrier
-    // or commits.  Two issuers on different SM sub-partitions therefore take
-    // alternate blocks: issuer i runs group j (PV_j, then S_{j+3} into the
-    // buffer PV_j has just read) for j = i, i + 2, ...; while one waits, the
-    // other keeps the queue filled.  O is zeroed before the first PV, so the
-    // two issuers' PV MMAs may accumulate in either order.  Each group's
-    // commit frees both of its ring slots.
     const int me = warp == kMmaWarp ? 0 : 1;
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, D, 1);
-      constexpr uint32_t kSlotStep = L::kTileBytes >> 4;  // descriptor units per slot
-      const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
+      constexpr uint32_t kBufStep = L::kTileBytes >> 4;  // descriptor units per buffer
+      const uint64_t dq = smem_desc_sw128(sQ(0), 16, 1024);
       const uint64_t dk = smem_desc_sw128(sSlot(0), 16, 1024);
       const uint64_t dv = smem_desc_sw128(sSlot(0), L::kChunkBytes, 1024);
-      const int n0 = n < 3 ? n : 3;
       bool ok = true;
       auto wait_pos = [&](int pos) {
-        ok = ok && mbar_wait(&bars.full[pos % NS], (pos / NS) & 1, abort_flag, dev_status, 0x2, kWaitNs);
+        ok = ok && mbar_wait(&bars.full[pos % NS], (pos / NS) & 1, abort_flag, dev_status, 0x2,
+                             kWaitNs);
       };
-      auto mma_s = [&](int jj, int kslot, int kk) {
-        const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-        mma_ss(tmem + (jj % 3) * 128, dq + off, dk + static_cast<uint64_t>(kslot * kSlotStep) + off,
-               idesc_s, kk > 0 ? 1u : 0u);
+      // S_J = Q(tile k) K^T, K from ring position pos, into score buffer J mod 3
+      auto issue_s = [&](int J, int k, int pos) {
+        const uint64_t dqs = dq + static_cast<uint64_t>((k & 1) * kBufStep);
+        const uint64_t dks = dk + static_cast<uint64_t>((pos % NS) * kBufStep);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + (J % 3) * 128, dqs + off, dks + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
       };
-      if (me == 0) {
-        // prologue: S_0 .. S_{n0-1}
-        ok = mbar_wait(&bars.q_full, 0, abort_flag, dev_status, 0x2, kWaitNs);
-        for (int jj = 0; jj < n0 && ok; ++jj) {
-          wait_pos(jj);
+      int last1 = -1, last2 = -1;  // last two groups of the previous non-empty tile
+      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
+        if (c.n == 0) continue;
+        const int n0 = c.n < 3 ? c.n : 3;
+        const int nk = c.n > 3 ? c.n - 3 : 0;
+        if (me == 0) {
+          // prologue: the score buffers are free once the previous tile's MMAs are done
+          ok = mbar_wait(&bars.q_full[c.k & 1], (c.k >> 1) & 1, abort_flag, dev_status, 0x2,
+                         kWaitNs);
+          if (ok && last1 >= 0) ok = wait_group(bars.rel, last1, abort_flag, dev_status);
+          if (ok && last2 >= 0) ok = wait_group(bars.rel, last2, abort_flag, dev_status);
+          for (int jj = 0; jj < n0 && ok; ++jj) {
+            wait_pos(c.pos0 + jj);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(c.J0 + jj, c.k, c.pos0 + jj);
+            mma_commit(&bars.s_full[(c.J0 + jj) % 3]);
+          }
           if (!ok) break;
+          mma_commit(&bars.rel[group_of_prologue(c) % kRel]);
+        }
+        for (int j = ((c.J0 & 1) == me) ? 0 : 1; j < c.n && ok; j += 2) {
+          const int J = c.J0 + j;
+          ok = mbar_wait(&bars.p_full[J % 3], (J / 3) & 1, abort_flag, dev_status, 0x2, kWaitNs);
+          const int pv = c.pos0 + n0 + j + (j < nk ? j : nk);
+          const bool more = j + 3 < c.n;
+          wait_pos(pv);
+          if (more) wait_pos(pv + 1);
+          if (!ok) break;
+          const uint64_t dvs = dv + static_cast<uint64_t>((pv % NS) * kBufStep);
+          const uint32_t a_col = tmem + (J % 3) * 128;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) mma_s(jj, jj % NS, kk);
-          mma_commit(&bars.s_full[jj]);
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + kColO, a_col + kk * 8, dvs + static_cast<uint64_t>(kk * (2048 >> 4)),
+                   idesc_pv, 1u);
+          if (more) {
+            // buffer J mod 3 is free once PV_J has read P_J (this issuer's MMAs run in order)
+            issue_s(J + 3, c.k, pv + 1);
+            mma_commit(&bars.s_full[J % 3]);
+          }
+          mma_commit(&bars.rel[group_of_block(c, j) % kRel]);
         }
-        mma_commit(&bars.pro_done);
+        last1 = group_of_block(c, c.n - 1);
+        last2 = c.n >= 2 ? group_of_block(c, c.n - 2) : -1;
       }
-      // (issuer 1 needs no prologue wait: P_1 exists only after S_1 and Q were used)
-      for (int j = me; j < n && ok; j += 2) {
-        ok = mbar_wait(&bars.p_full[j % 3], (j / 3) & 1, abort_flag, dev_status, 0x2, kWaitNs);
-        const int pv = ring_pos_v(j, n);
-        const bool more = j + 3 < n;
-        wait_pos(pv);
-        if (more) wait_pos(pv + 1);
-        if (!ok) break;
-        const uint64_t dvs = dv + static_cast<uint64_t>((pv % NS) * kSlotStep);
-        const uint32_t a_col = tmem + (j % 3) * 128;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + L::kColO, a_col + kk * 8, dvs + static_cast<uint64_t>(kk * (2048 >> 4)),
-                 idesc_pv, 1u);
-        if (more) {
-          // buffer j mod 3 is free once PV_j has read P_j (one issuer's MMAs run in order)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) mma_s(j + 3, (pv + 1) % NS, kk);
-          mma_commit(&bars.s_full[j % 3]);
-        }
-        mma_commit(&bars.rel[j & 7]);
-      }
-      mma_commit(&bars.o_done);
       mma_commit(&bars.drain);
       mbar_drain(&bars.drain, 0, kDrainNs);
     }
     __syncwarp();
   } else {
     // ================================================================ softmax
-    const int g = warp >> 2;  // group: blocks j = g, g + 2, ...
+    const int g = warp >> 2;  // group: blocks with J % 2 == g
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t o_addr = tmem + lane_off + L::kColO;
-    const int grow = qb * kTile + row;
-    const float c = args.scale_log2;
-    float m_own = -INFINITY;  // reference of this group's l_sum
-    float l0 = 0.f, l1 = 0.f;
+    const uint32_t o_addr = tmem + lane_off + kColO;
+    const float csc = args.scale_log2;
     bool good = true;
 
-    for (int j = g; j < n && good; j += 2) {
-      const int kb = __ldg(list + j);
-      const int buf = j % 3;
-      const uint32_t s_addr = tmem + lane_off + buf * 128;
-      if (!warp_wait(&bars.s_full[buf], (j / 3) & 1, abort_flag, dev_status)) { good = false; break; }
-      tc_fence_after();
-      float x[kTile];
-      {
-        uint32_t sr[kTile];
-        tmem_ld128_wait(s_addr, sr);
-#pragma unroll
-        for (int k = 0; k < kTile; ++k) x[k] = __uint_as_float(sr[k]);
-      }
-      int valid = kTile;
-      if (kb < 0 || kb >= args.nkb) {
-        valid = 0;
-        if (row == 0 && dev_status) atomicOr(dev_status, 0x1);
-      } else if ((kb + 1) * kTile > args.Lkv) {
-        valid = args.Lkv - kb * kTile;
-      }
-      if (valid < kTile) {
-#pragma unroll
-        for (int k = 0; k < kTile; ++k)
-          if (k >= valid) x[k] = -INFINITY;
-      }
-      float mx0 = fmaxf(x[0], x[4]), mx1 = fmaxf(x[1], x[5]);
-      float mx2 = fmaxf(x[2], x[6]), mx3 = fmaxf(x[3], x[7]);
-#pragma unroll
-      for (int k = 8; k < kTile; k += 8) {
-        mx0 = max3(mx0, x[k], x[k + 4]);
-        mx1 = max3(mx1, x[k + 1], x[k + 5]);
-        mx2 = max3(mx2, x[k + 2], x[k + 6]);
-        mx3 = max3(mx3, x[k + 3], x[k + 7]);
-      }
-      const float bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;  // block row max
-      // provisional reference: the shared one, raised to bm if bm is far above it
-      const float m_cur = m_sh[row];
-      const float m_use = (m_cur == -INFINITY || bm > m_cur + kLazyRescale) ? bm : m_cur;
-      const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
-      float lb0 = 0.f, lb1 = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float p0 = ex2_approx(fmaf(x[cc * 32 + 2 * k], c, neg));
-          const float p1 = ex2_approx(fmaf(x[cc * 32 + 2 * k + 1], c, neg));
-          lb0 += p0;
-          lb1 += p1;
-          pk[k] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(s_addr + cc * 16, pk);
-      }
-      float lb = lb0 + lb1;
-
-      // ---- finalise block j in block order
-      if (j > 0) {
-        const int pj = j - 1;
-        if (!warp_wait(&bars.p_full[pj % 3], (pj / 3) & 1, abort_flag, dev_status)) { good = false; break; }
-      }
-      const float m_fin = m_sh[row];
-      const bool raise = m_fin == -INFINITY ? (bm != -INFINITY) : (bm > m_fin + kLazyRescale);
-      const float m_blk = raise ? bm : m_fin;  // reference of block j from now on
-      // O holds non-zero values only once some earlier block had a finite reference
-      const bool o_live = raise && m_fin != -INFINITY;
-      if (__any_sync(0xffffffffu, o_live)) {
-        // PV_{j-1} must have completed before O is rewritten
-        // every earlier PV is complete once groups j-1 and j-2 (the latest of each
-        // issuer) have released their ring slots
-        const int pj = j - 1;
-        if (!warp_wait(&bars.rel[pj & 7], (pj >> 3) & 1, abort_flag, dev_status)) { good = false; break; }
-        if (pj >= 1 &&
-            !warp_wait(&bars.rel[(pj - 1) & 7], ((pj - 1) >> 3) & 1, abort_flag, dev_status)) {
+    for (TileCursor c = first; c.t < total; cursor_next(c, args, total, threadIdx.x == 0)) {
+      float m_own = -INFINITY;  // reference of this group's row sum
+      float l_own = 0.f;
+      for (int j = ((c.J0 & 1) == g) ? 0 : 1; j < c.n && good; j += 2) {
+        const int J = c.J0 + j;
+        const int kb = __ldg(c.list + j);
+        const int buf = J % 3;
+        const uint32_t s_addr = tmem + lane_off + buf * 128;
+        if (!warp_wait(&bars.s_full[buf], (J / 3) & 1, abort_flag, dev_status)) {
           good = false;
           break;
         }
         tc_fence_after();
-        const float alpha = o_live ? ex2_approx(m_fin - bm) : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t orr[32];
-          tmem_ld32_wait(o_addr + cc * 32, orr);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
-          tmem_st32(o_addr + cc * 32, orr);
+        int valid = kTile;
+        if (kb < 0 || kb >= args.nkb) {
+          valid = 0;
+          if (row == 0 && dev_status) atomicOr(dev_status, 0x1);
+        } else if ((kb + 1) * kTile > args.Lkv) {
+          valid = args.Lkv - kb * kTile;
         }
-      }
-      const bool fix_p = (m_use != m_blk) && m_use != -INFINITY;
-      if (__any_sync(0xffffffffu, fix_p)) {
-        // the shared reference moved while P_j was computed: rescale P_j to m_blk
-        tmem_wait_st();
-        const float beta = fix_p ? ex2_approx(m_use - m_blk) : 1.f;
-        if (fix_p) lb *= beta;
+        // pass 1: the block's row max
+        float bm;
+        {
+          uint32_t sr[kTile];
+          tmem_ld128_wait(s_addr, sr);
+          float x[kTile];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t pr[32];
-          tmem_ld32_wait(s_addr + cc * 32, pr);
+          for (int k = 0; k < kTile; ++k) x[k] = __uint_as_float(sr[k]);
+          if (valid < kTile) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float lo = __uint_as_float(pr[k] << 16) * beta;
-            const float hi = __uint_as_float(pr[k] & 0xffff0000u) * beta;
-            pr[k] = pack_bf16x2(lo, hi);
+            for (int k = 0; k < kTile; ++k)
+              if (k >= valid) x[k] = -INFINITY;
           }
-          tmem_st32(s_addr + cc * 32, pr);
+          float mx0 = fmaxf(x[0], x[4]), mx1 = fmaxf(x[1], x[5]);
+          float mx2 = fmaxf(x[2], x[6]), mx3 = fmaxf(x[3], x[7]);
+#pragma unroll
+          for (int k = 8; k < kTile; k += 8) {
+            mx0 = max3(mx0, x[k], x[k + 4]);
+            mx1 = max3(mx1, x[k + 1], x[k + 5]);
+            mx2 = max3(mx2, x[k + 2], x[k + 6]);
+            mx3 = max3(mx3, x[k + 3], x[k + 7]);
+          }
+          bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * csc;
         }
-      }
-      if (raise) m_sh[row] = m_blk;
-      // this group's running sum, moved to the block's reference
-      if (m_blk != m_own) {
-        const float f = (m_own == -INFINITY) ? 0.f : ex2_approx(m_own - m_blk);
-        l0 *= f;
-        l1 *= f;
-        m_own = m_blk;
-      }
-      l0 += lb;
-      if (j == 0) {
-        // O starts at zero: PV MMAs of the two issuers accumulate in either order
-        uint32_t zr[32];
+        // provisional reference: the shared one, raised to bm if bm is far above it
+        const float m_cur = m_sh[row];
+        const float m_use = (m_cur == -INFINITY || bm > m_cur + kLazyRescale) ? bm : m_cur;
+        const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
+        // pass 2: P = 2^(s * scale - m) in packed pairs, S re-read 32 columns at a time
+        // (the next chunk's load overlaps this chunk's math; P chunk cc overwrites
+        // columns [16cc, 16cc + 16), already read).  The pairs kPolyPairs selects take
+        // the FMA-pipe exponential, the rest the MUFU one, so neither unit limits the block.
+        const uint64_t sc2 = f2_pack(csc, csc), neg2 = f2_pack(neg, neg);
+        uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
+        uint32_t sa[32], sb[32];
+        tmem_ld32_async(s_addr, sa, __float_as_uint(neg));  // after pass 1's registers are free
 #pragma unroll
-        for (int k = 0; k < 32; ++k) zr[k] = 0u;
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&cur)[32] = (cc & 1) ? sb : sa;
+          uint32_t(&nxt)[32] = (cc & 1) ? sa : sb;
+          tmem_wait_ld_tied(cur);
+          if (cc < 3) tmem_ld32_async(s_addr + (cc + 1) * 32, nxt);
+          if (valid < kTile) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) tmem_st32(o_addr + cc * 32, zr);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars.p_full[buf]);
-    }
+            for (int k = 0; k < 32; ++k)
+              if (cc * 32 + k >= valid) cur[k] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            float e0, e1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(cur[2 * k]), __uint_as_float(cur[2 * k + 1])),
+                             sc2, neg2),
+                      e0, e1);
+            if ((kPolyPairs >> k) & 1u) {
+              exp2_poly2(e0, e1, p0, p1);
+            } else {
+              p0 = ex2_approx(e0);
+              p1 = ex2_approx(e1);
+            }
+            if (k & 1) {
+              acc1 = f2_add(acc1, f2_pack(p0, p1));
+            } else {
+              acc0 = f2_add(acc0, f2_pack(p0, p1));
+            }
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_addr + cc * 16, pk);
+        }
+        float lb;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(acc0, acc1), a0, a1);
+          lb = a0 + a1;
+        }
 
-    // ---- epilogue: both groups' sums against the final reference.  Once o_done
-    // has fired every MMA has finished and every TMA load has landed, so the
-    // first ring slot is free for the exchange.
-    if (good && n > 0) good = warp_wait(&bars.o_done, 0, abort_flag, dev_status);
-    float* merge_m = reinterpret_cast<float*>(smem_raw + (smem_base - smem_addr(smem_raw)) + L::kRing);
-    float* merge_l = merge_m + 2 * kTile;
-    merge_m[g * kTile + row] = m_own;
-    merge_l[g * kTile + row] = l0 + l1;
-    tc_fence_before();
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    tc_fence_after();
-    const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
-    if (!aborted) {
-      const float m = m_sh[row];
-      const float ma = merge_m[row], mb = merge_m[kTile + row];
-      const float sa = (ma == -INFINITY) ? 0.f : ex2_approx(ma - m);
-      const float sb = (mb == -INFINITY) ? 0.f : ex2_approx(mb - m);
-      const float l = merge_l[row] * sa + merge_l[kTile + row] * sb;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = args.o + b * args.o_sb + h * args.o_sh + grow * args.o_sr;
-      // group 0 writes columns [0, D/2), group 1 writes [D/2, D)
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int col = g * (D / 2) + cc * 32;
-        uint32_t ro[32];
-        if (n > 0) {
-          tmem_ld32_wait(o_addr + col, ro);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) ro[k] = 0u;
+        // ---- finalise block J in sequence order
+        if (J > 0 &&
+            !warp_wait(&bars.p_full[(J - 1) % 3], ((J - 1) / 3) & 1, abort_flag, dev_status)) {
+          good = false;
+          break;
         }
-        uint32_t pk[16];
+        const float m_fin = m_sh[row];
+        const bool raise = m_fin == -INFINITY ? (bm != -INFINITY) : (bm > m_fin + kLazyRescale);
+        const float m_blk = raise ? bm : m_fin;  // reference of block J from now on
+        // O holds non-zero values only once an earlier block of the tile had a finite reference
+        const bool o_live = raise && m_fin != -INFINITY;
+        if (__any_sync(0xffffffffu, o_live)) {
+          // every earlier PV of the tile is complete once the latest group of each
+          // issuer (blocks j-1 and j-2) has completed
+          if (!warp_wait_group(bars.rel, group_of_block(c, j - 1), abort_flag, dev_status) ||
+              (j >= 2 &&
+               !warp_wait_group(bars.rel, group_of_block(c, j - 2), abort_flag, dev_status))) {
+            good = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = o_live ? ex2_approx(m_fin - bm) : 1.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pk[k] = pack_bf16x2(__uint_as_float(ro[2 * k]) * inv_l,
-                              __uint_as_float(ro[2 * k + 1]) * inv_l);
-        if (grow < args.Lq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + col);
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t orr[32];
+            tmem_ld32_wait(o_addr + cc * 32, orr);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int k = 0; k < 32; ++k) orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
+            tmem_st32(o_addr + cc * 32, orr);
+          }
+        }
+        const bool fix_p = (m_use != m_blk) && m_use != -INFINITY;
+        if (__any_sync(0xffffffffu, fix_p)) {
+          // the shared reference moved while P_J was computed: rescale P_J to m_blk
+          tmem_wait_st();
+          const float beta = fix_p ? ex2_approx(m_use - m_blk) : 1.f;
+          if (fix_p) lb *= beta;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t pr[32];
+            tmem_ld32_wait(s_addr + cc * 32, pr);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float lo = __uint_as_float(pr[k] << 16) * beta;
+              const float hi = __uint_as_float(pr[k] & 0xffff0000u) * beta;
+              pr[k] = pack_bf16x2(lo, hi);
+            }
+            tmem_st32(s_addr + cc * 32, pr);
+          }
+        }
+        if (raise) m_sh[row] = m_blk;
+        // this group's running sum, moved to the block's reference
+        if (m_blk != m_own) {
+          l_own *= (m_own == -INFINITY) ? 0.f : ex2_approx(m_own - m_blk);
+          m_own = m_blk;
+        }
+        l_own += lb;
+        if (j == 0) {
+          // O starts at zero: the two issuers' PV MMAs accumulate in either order
+          uint32_t zr[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) zr[k] = 0u;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_st32(o_addr + cc * 32, zr);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars.p_full[buf]);
+      }
+
+      // ---- epilogue of the tile
+      if (good && c.n > 0) {
+        good = warp_wait_group(bars.rel, group_of_block(c, c.n - 1), abort_flag, dev_status) &&
+               (c.n < 2 ||
+                warp_wait_group(bars.rel, group_of_block(c, c.n - 2), abort_flag, dev_status));
+      }
+      // every MMA of the tile is done: its Q buffer holds the two groups' sums
+      float* xch = reinterpret_cast<float*>(smem_gen + L::kQ + (c.k & 1) * L::kTileBytes);
+      if (c.n > 0) {
+        xch[g * kTile + row] = m_own;
+        xch[(2 + g) * kTile + row] = l_own;
+      }
+      tc_fence_before();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      tc_fence_after();
+      const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
+      if (!aborted) {
+        float l = 0.f, m = -INFINITY, inv_l = 0.f;
+        if (c.n > 0) {
+          m = m_sh[row];
+          const float ma = xch[row], mb = xch[kTile + row];
+          const float sa = (ma == -INFINITY) ? 0.f : ex2_approx(ma - m);
+          const float sb = (mb == -INFINITY) ? 0.f : ex2_approx(mb - m);
+          l = xch[2 * kTile + row] * sa + xch[3 * kTile + row] * sb;
+          inv_l = l > 0.f ? 1.f / l : 0.f;
+        }
+        const TileCoord tc = tile_coord(c.t, args);
+        const int grow = tc.qb * kTile + row;
+        __nv_bfloat16* orow = args.o + tc.b * args.o_sb + tc.h * args.o_sh + grow * args.o_sr;
+        // group 0 writes columns [0, D/2), group 1 writes [D/2, D)
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          const int col = g * (D / 2) + cc * 32;
+          uint32_t ro[32];
+          if (c.n > 0) {
+            tmem_ld32_wait(o_addr + col, ro);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ro[k] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack_bf16x2(__uint_as_float(ro[2 * k]) * inv_l,
+                                __uint_as_float(ro[2 * k + 1]) * inv_l);
+          if (grow < args.Lq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (g == 0 && args.lse && grow < args.Lq) {
+          args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.Lq + grow] =
+              l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
       }
-      if (g == 0 && args.lse && grow < args.Lq) {
-        args.lse[(static_cast<int64_t>(b) * args.H + h) * args.Lq + grow] =
-            l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
-      }
+      // both groups are done with m, the exchanged sums and O: reset m, then hand
+      // the Q buffer back to the producer (its next writes come through TMA)
+      fence_proxy_async_smem();
+      tc_fence_before();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (g == 0) m_sh[row] = -INFINITY;
+      if (threadIdx.x == 0 && c.n > 0) mbar_arrive(&bars.epi[c.k & 1]);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      tc_fence_after();
     }
   }
 

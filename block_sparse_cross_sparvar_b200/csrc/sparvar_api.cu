@@ -139,8 +139,18 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-  dim3 grid(a.nqb, a.H, a.B);
-  kern<<<grid, sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, a);
+  // persistent: one CTA per SM, each walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
+  const int64_t tiles = static_cast<int64_t>(a.B) * a.H * a.nqb;
+  const int64_t grid = tiles < sms ? tiles : sms;
+  // the kernel's per-CTA sequence counters (blocks, ring positions) are 32-bit
+  if (ceil_div(tiles, grid) * (3 * static_cast<int64_t>(a.idx_row_len) + 1) >= (int64_t{1} << 31))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %d too large per SM",
+                static_cast<long long>(tiles), a.idx_row_len);
+  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return SPARVAR_OK;
@@ -264,6 +274,8 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
     return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
   if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
     return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  if (static_cast<int64_t>(B) * H * ceil_div(Lq, 128) > (int64_t{1} << 30))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "B*H*ceil(Lq/128) above 2^30 query tiles");
   int rc;
   if ((rc = check_operand(q, q_strides, B, H, Lq, D, "q"))) return rc;
   if ((rc = check_operand(k, k_strides, B, H, Lkv, D, "k"))) return rc;
