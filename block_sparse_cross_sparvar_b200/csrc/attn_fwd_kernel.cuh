@@ -387,53 +387,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if ((kb + 1) * kTile > args.Lkv) {
           valid = args.Lkv - kb * kTile;
         }
-        // pass 1: the block's row max
+        // pass 1: the block's row max.  Columns 0-63 stay in registers for pass 2.
         float bm;
+        uint32_t s0[32], s1[32];
         {
           uint32_t sr[kTile];
           tmem_ld128_wait(s_addr, sr);
-          float x[kTile];
-#pragma unroll
-          for (int k = 0; k < kTile; ++k) x[k] = __uint_as_float(sr[k]);
           if (valid < kTile) {
 #pragma unroll
             for (int k = 0; k < kTile; ++k)
-              if (k >= valid) x[k] = -INFINITY;
+              if (k >= valid) sr[k] = __float_as_uint(-INFINITY);
           }
-          float mx0 = fmaxf(x[0], x[4]), mx1 = fmaxf(x[1], x[5]);
-          float mx2 = fmaxf(x[2], x[6]), mx3 = fmaxf(x[3], x[7]);
+          float mx0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[4]));
+          float mx1 = fmaxf(__uint_as_float(sr[1]), __uint_as_float(sr[5]));
+          float mx2 = fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[6]));
+          float mx3 = fmaxf(__uint_as_float(sr[3]), __uint_as_float(sr[7]));
 #pragma unroll
           for (int k = 8; k < kTile; k += 8) {
-            mx0 = max3(mx0, x[k], x[k + 4]);
-            mx1 = max3(mx1, x[k + 1], x[k + 5]);
-            mx2 = max3(mx2, x[k + 2], x[k + 6]);
-            mx3 = max3(mx3, x[k + 3], x[k + 7]);
+            mx0 = max3(mx0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 4]));
+            mx1 = max3(mx1, __uint_as_float(sr[k + 1]), __uint_as_float(sr[k + 5]));
+            mx2 = max3(mx2, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 6]));
+            mx3 = max3(mx3, __uint_as_float(sr[k + 3]), __uint_as_float(sr[k + 7]));
           }
           bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * csc;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            s0[k] = sr[k];
+            s1[k] = sr[32 + k];
+          }
         }
         // provisional reference: the shared one, raised to bm if bm is far above it
         const float m_cur = m_sh[row];
         const float m_use = (m_cur == -INFINITY || bm > m_cur + kLazyRescale) ? bm : m_cur;
         const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
-        // pass 2: P = 2^(s * scale - m) in packed pairs, S re-read 32 columns at a time
-        // (the next chunk's load overlaps this chunk's math; P chunk cc overwrites
-        // columns [16cc, 16cc + 16), already read).  The pairs kPolyPairs selects take
-        // the FMA-pipe exponential, the rest the MUFU one, so neither unit limits the block.
+        // pass 2: P = 2^(s * scale - m) in packed pairs.  Columns 64-127 are re-read
+        // 32 at a time while the columns held in registers are worked on; P chunk cc
+        // (packed bf16) overwrites TMEM columns [16cc, 16cc + 16), already read.  The
+        // pairs kPolyPairs selects take the FMA-pipe exponential, the others the MUFU one.
         const uint64_t sc2 = f2_pack(csc, csc), neg2 = f2_pack(neg, neg);
         uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
-        uint32_t sa[32], sb[32];
-        tmem_ld32_async(s_addr, sa, __float_as_uint(neg));  // after pass 1's registers are free
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t(&cur)[32] = (cc & 1) ? sb : sa;
-          uint32_t(&nxt)[32] = (cc & 1) ? sa : sb;
-          tmem_wait_ld_tied(cur);
-          if (cc < 3) tmem_ld32_async(s_addr + (cc + 1) * 32, nxt);
-          if (valid < kTile) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (cc * 32 + k >= valid) cur[k] = __float_as_uint(-INFINITY);
-          }
+        auto p_chunk = [&](const uint32_t(&cur)[32], int cc) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -455,6 +448,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_addr + cc * 16, pk);
+        };
+        auto mask_chunk = [&](uint32_t(&cur)[32], int cc) {
+          if (valid < kTile) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (cc * 32 + k >= valid) cur[k] = __float_as_uint(-INFINITY);
+          }
+        };
+        {
+          uint32_t s2[32];
+          tmem_ld32_async(s_addr + 64, s2, __float_as_uint(neg));
+          p_chunk(s0, 0);
+          p_chunk(s1, 1);
+          tmem_wait_ld_tied(s2);
+          uint32_t s3[32];
+          tmem_ld32_async(s_addr + 96, s3, s2[0]);
+          mask_chunk(s2, 2);
+          p_chunk(s2, 2);
+          tmem_wait_ld_tied(s3);
+          mask_chunk(s3, 3);
+          p_chunk(s3, 3);
         }
         float lb;
         {
