@@ -36,10 +36,14 @@
 // m (block max more than 2^8 above it: O is rescaled in place once the tile's
 // earlier PVs have completed) or, if m moved meanwhile, rescales its own P in
 // TMEM.  O is zeroed before a tile's first PV, so the two issuers' PVs may
-// accumulate in either order.  The epilogue waits for the tile's last two
-// groups, merges the two groups' row sums against the final m (exchanging them
-// through the tile's Q buffer, which no MMA reads any more), writes O and the
-// LSE, and hands the Q buffer back to the producer.
+// accumulate in either order.  Each block's softmax takes two passes over S in
+// TMEM: the row max, then P in packed f32x2 arithmetic from the 96 columns kept
+// in registers plus the last 32 re-read.  The epilogue waits for the tile's
+// last two groups, merges the two groups' row sums against the final m
+// (exchanging them through the tile's Q buffer, which no MMA reads any more),
+// stages the normalised bf16 output in that buffer in the output tensor map's
+// swizzled layout, sends it with one TMA store per 64 columns, writes the LSE,
+// and hands the buffer back to the producer once the store has read it.
 #pragma once
 
 #include <cuda.h>
@@ -172,7 +176,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Args args) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Args args) {
   using L = Layout<D>;
   constexpr int NS = L::kSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -215,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -387,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if ((kb + 1) * kTile > args.Lkv) {
           valid = args.Lkv - kb * kTile;
         }
-        // pass 1: the block's row max.  Columns 0-63 stay in registers for pass 2.
+        // pass 1: the block's row max.  Columns 0-95 stay in registers for pass 2.
         float bm;
-        uint32_t s0[32], s1[32];
+        uint32_t s0[32], s1[32], s2[32];
         {
           uint32_t sr[kTile];
           tmem_ld128_wait(s_addr, sr);
@@ -414,16 +420,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 32; ++k) {
             s0[k] = sr[k];
             s1[k] = sr[32 + k];
+            s2[k] = sr[64 + k];
           }
         }
         // provisional reference: the shared one, raised to bm if bm is far above it
         const float m_cur = m_sh[row];
         const float m_use = (m_cur == -INFINITY || bm > m_cur + kLazyRescale) ? bm : m_cur;
         const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
-        // pass 2: P = 2^(s * scale - m) in packed pairs.  Columns 64-127 are re-read
-        // 32 at a time while the columns held in registers are worked on; P chunk cc
-        // (packed bf16) overwrites TMEM columns [16cc, 16cc + 16), already read.  The
-        // pairs kPolyPairs selects take the FMA-pipe exponential, the others the MUFU one.
+        // pass 2: P = 2^(s * scale - m) in packed pairs.  Columns 96-127 are re-read
+        // while the columns held in registers are worked on; P chunk cc (packed bf16)
+        // overwrites TMEM columns [16cc, 16cc + 16), already read.  The pairs
+        // kPolyPairs selects take the FMA-pipe exponential, the others the MUFU one.
         const uint64_t sc2 = f2_pack(csc, csc), neg2 = f2_pack(neg, neg);
         uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
         auto p_chunk = [&](const uint32_t(&cur)[32], int cc) {
@@ -457,14 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         {
-          uint32_t s2[32];
-          tmem_ld32_async(s_addr + 64, s2, __float_as_uint(neg));
+          uint32_t s3[32];
+          tmem_ld32_async(s_addr + 96, s3, __float_as_uint(neg));
           p_chunk(s0, 0);
           p_chunk(s1, 1);
-          tmem_wait_ld_tied(s2);
-          uint32_t s3[32];
-          tmem_ld32_async(s_addr + 96, s3, s2[0]);
-          mask_chunk(s2, 2);
           p_chunk(s2, 2);
           tmem_wait_ld_tied(s3);
           mask_chunk(s3, 3);
@@ -553,8 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                (c.n < 2 ||
                 warp_wait_group(bars.rel, group_of_block(c, c.n - 2), abort_flag, dev_status));
       }
-      // every MMA of the tile is done: its Q buffer holds the two groups' sums
-      float* xch = reinterpret_cast<float*>(smem_gen + L::kQ + (c.k & 1) * L::kTileBytes);
+      // every MMA of the tile is done and its Q buffer is free: it takes first the two
+      // groups' sums, then the bf16 output tile, which leaves through a TMA store
+      uint8_t* qbuf = smem_gen + L::kQ + (c.k & 1) * L::kTileBytes;
+      float* xch = reinterpret_cast<float*>(qbuf);
       if (c.n > 0) {
         xch[g * kTile + row] = m_own;
         xch[(2 + g) * kTile + row] = l_own;
@@ -563,59 +568,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       tc_fence_after();
       const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
-      if (!aborted) {
-        float l = 0.f, m = -INFINITY, inv_l = 0.f;
-        if (c.n > 0) {
-          m = m_sh[row];
-          const float ma = xch[row], mb = xch[kTile + row];
-          const float sa = (ma == -INFINITY) ? 0.f : ex2_approx(ma - m);
-          const float sb = (mb == -INFINITY) ? 0.f : ex2_approx(mb - m);
-          l = xch[2 * kTile + row] * sa + xch[3 * kTile + row] * sb;
-          inv_l = l > 0.f ? 1.f / l : 0.f;
-        }
-        const TileCoord tc = tile_coord(c.t, args);
-        const int grow = tc.qb * kTile + row;
-        __nv_bfloat16* orow = args.o + tc.b * args.o_sb + tc.h * args.o_sh + grow * args.o_sr;
-        // group 0 writes columns [0, D/2), group 1 writes [D/2, D)
-#pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
-          const int col = g * (D / 2) + cc * 32;
-          uint32_t ro[32];
-          if (c.n > 0) {
-            tmem_ld32_wait(o_addr + col, ro);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) ro[k] = 0u;
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pk[k] = pack_bf16x2(__uint_as_float(ro[2 * k]) * inv_l,
-                                __uint_as_float(ro[2 * k + 1]) * inv_l);
-          if (grow < args.Lq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
-        }
-        if (g == 0 && args.lse && grow < args.Lq) {
-          args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.Lq + grow] =
-              l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
-        }
+      const TileCoord tc = tile_coord(c.t, args);
+      const int grow = tc.qb * kTile + row;
+      float l = 0.f, m = -INFINITY, inv_l = 0.f;
+      if (c.n > 0) {
+        m = m_sh[row];
+        const float ma = xch[row], mb = xch[kTile + row];
+        const float sa = (ma == -INFINITY) ? 0.f : ex2_approx(ma - m);
+        const float sb = (mb == -INFINITY) ? 0.f : ex2_approx(mb - m);
+        l = xch[2 * kTile + row] * sa + xch[3 * kTile + row] * sb;
+        inv_l = l > 0.f ? 1.f / l : 0.f;
       }
-      // both groups are done with m, the exchanged sums and O: reset m, then hand
-      // the Q buffer back to the producer (its next writes come through TMA)
-      fence_proxy_async_smem();
-      tc_fence_before();
+      if (!aborted && g == 0 && args.lse && grow < args.Lq) {
+        args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.Lq + grow] =
+            l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      }
+      if (c.n > 0) {
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the sums are read: reuse the buffer
+        if (!aborted) {
+          // row `row`, columns [g D/2, (g+1) D/2), into the 128B-swizzled layout of the
+          // output tensor map: 64-column chunks of 128 rows x 128 bytes, 16-byte unit u of
+          // row r at position u ^ (r mod 8)
+#pragma unroll
+          for (int cc = 0; cc < D / 64; ++cc) {
+            const int col = g * (D / 2) + cc * 32;
+            uint32_t ro[32];
+            tmem_ld32_wait(o_addr + col, ro);
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              pk[k] = pack_bf16x2(__uint_as_float(ro[2 * k]) * inv_l,
+                                  __uint_as_float(ro[2 * k + 1]) * inv_l);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int cv = col + 8 * v;
+              const int unit = (cv & 63) >> 3;
+              uint4* dst = reinterpret_cast<uint4*>(qbuf + (cv >> 6) * L::kChunkBytes + row * 128 +
+                                                    ((unit ^ (row & 7)) << 4));
+              *dst = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (threadIdx.x == 0 && !aborted) {
+#pragma unroll
+          for (int ch = 0; ch < L::kChunks; ++ch)
+            tma_store_4d(&tm_o, sQ(c.k) + ch * L::kChunkBytes, ch * 64, tc.qb * kTile, tc.h, tc.b);
+          bulk_commit_group();
+        }
+      } else if (!aborted && grow < args.Lq) {
+        // empty list: zero rows (the Q buffer may already hold the next tile's Q)
+        __nv_bfloat16* orow = args.o + tc.b * args.o_sb + tc.h * args.o_sh + grow * args.o_sr;
+#pragma unroll
+        for (int v = 0; v < D / 16; ++v)
+          reinterpret_cast<uint4*>(orow + g * (D / 2))[v] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      // reset m for the next tile once everyone has read it
       asm volatile("bar.sync 1, 256;" ::: "memory");
       if (g == 0) m_sh[row] = -INFINITY;
-      if (threadIdx.x == 0 && c.n > 0) mbar_arrive(&bars.epi[c.k & 1]);
       asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0 && c.n > 0) {
+        bulk_wait_read_all();  // the output tile has left the buffer: hand it back
+        mbar_arrive(&bars.epi[c.k & 1]);
+      }
       tc_fence_after();
     }
   }
 
+  if (threadIdx.x == 0) bulk_wait_all();  // output stores complete before the CTA exits
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -133,7 +133,7 @@ int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 template <int D>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const sparvar::fwd::Args& a, cudaStream_t stream) {
+                      const CUtensorMap& to, const sparvar::fwd::Args& a, cudaStream_t stream) {
   auto kern = sparvar::fwd::attn_fwd_kernel<D>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -150,7 +150,7 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   if (ceil_div(tiles, grid) * (3 * static_cast<int64_t>(a.idx_row_len) + 1) >= (int64_t{1} << 31))
     return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %d too large per SM",
                 static_cast<long long>(tiles), a.idx_row_len);
-  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, a);
+  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return SPARVAR_OK;
@@ -302,13 +302,14 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   a.lse = lse;
   a.dev_status = dev_status;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
   if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
   if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
+  if ((rc = make_tmap(&to, o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o"))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_fwd_kernel<128>(tq, tk, tv, a, st);
-  return launch_fwd_kernel<64>(tq, tk, tv, a, st);
+  if (D == 128) return launch_fwd_kernel<128>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
