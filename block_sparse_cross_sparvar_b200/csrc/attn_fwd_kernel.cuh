@@ -78,6 +78,8 @@ struct Args {
   const int32_t* kv_idx;
   int64_t list_sb, list_sh;
   int idx_row_len;
+  const uint64_t* tile_mask;  // per list entry, fine-block bits; null: whole tiles
+  int mask_shift;             // log2 of the fine block side (4, 5 or 6)
   __nv_bfloat16* o;
   int64_t o_sb, o_sh, o_sr;
   float* lse;  // [B][H][Lq] or null
@@ -393,16 +395,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if ((kb + 1) * kTile > args.Lkv) {
           valid = args.Lkv - kb * kTile;
         }
+        // with a fine block grid, bit i of `keep` keeps this row's columns
+        // [i << mask_shift, (i + 1) << mask_shift) of the tile
+        uint32_t keep = 0xffu;
+        bool fine = false;
+        if (args.tile_mask) {
+          const int fg = kTile >> args.mask_shift;
+          const uint32_t full = (1u << fg) - 1u;
+          const uint64_t mk = __ldg(args.tile_mask + (c.list - args.kv_idx) + j);
+          keep = static_cast<uint32_t>(mk >> ((row >> args.mask_shift) * fg)) & full;
+          fine = __any_sync(0xffffffffu, keep != full);
+          keep |= ~full;
+        }
+        auto dropped = [&](int col) {
+          return col >= valid || !((keep >> (col >> args.mask_shift)) & 1u);
+        };
         // pass 1: the block's row max.  Columns 0-95 stay in registers for pass 2.
         float bm;
         uint32_t s0[32], s1[32], s2[32];
         {
           uint32_t sr[kTile];
           tmem_ld128_wait(s_addr, sr);
-          if (valid < kTile) {
+          if (valid < kTile || fine) {
 #pragma unroll
             for (int k = 0; k < kTile; ++k)
-              if (k >= valid) sr[k] = __float_as_uint(-INFINITY);
+              if (dropped(k)) sr[k] = __float_as_uint(-INFINITY);
           }
           float mx0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[4]));
           float mx1 = fmaxf(__uint_as_float(sr[1]), __uint_as_float(sr[5]));
@@ -457,10 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(s_addr + cc * 16, pk);
         };
         auto mask_chunk = [&](uint32_t(&cur)[32], int cc) {
-          if (valid < kTile) {
+          if (valid < kTile || fine) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
-              if (cc * 32 + k >= valid) cur[k] = __float_as_uint(-INFINITY);
+              if (dropped(cc * 32 + k)) cur[k] = __float_as_uint(-INFINITY);
           }
         };
         {

@@ -2,9 +2,11 @@
 //   csla_mask_kernel      CSLA sink + cross-scale locality mask, one CTA per query block
 //   map_indices_kernel    CS4A proportional index mapping, one CTA per (b, h, dst query block)
 //   validate_lists_kernel range / order check of block lists, one warp per list
-// All three build a KV-block bitset in shared memory with atomicOr and then
-// compact it into an ascending list (-1 padded) with warp ballots.  Integer
-// only, so results are exact.
+//   coarsen_lists_kernel  fine (16/32/64) block lists -> 128x128 tile lists with
+//                         per-tile bitmasks, one CTA per (b, h, query tile)
+// They build a KV-block bitset in shared memory with atomicOr and then compact
+// it into an ascending list (-1 padded) with warp ballots.  Integer only, so
+// results are exact.
 #pragma once
 
 #include <cstdint>
@@ -173,6 +175,89 @@ __global__ void __launch_bounds__(kMaskThreads)
     compact_bitset(bits, d_nkb, d_idx + drow * d_nkb, d_cnt + drow,
                    d_mask ? d_mask + drow * d_nkb : nullptr);
   }
+}
+
+// ---------------------------------------------------------------- coarsening
+// Fine square blocks of side 128/g (g = 2, 4 or 8) grouped into 128x128 tiles.
+// For query tile T and KV tile kt, bit (qi * g + ki) of the tile mask is set
+// when fine KV block kt*g + ki is listed for fine query block T*g + qi; the tile
+// list holds, ascending, every kt whose mask is not zero.  Fine entries outside
+// [0, nkb_f) are flagged (SPARVAR_DEV_BAD_LIST) and skipped.  Dynamic shared
+// memory: nkt 64-bit masks, then ceil(nkt / 32) bitset words.
+__global__ void __launch_bounds__(kMaskThreads)
+    coarsen_lists_kernel(const int32_t* kv_cnt, const int32_t* kv_idx, int64_t l_sb, int64_t l_sh,
+                         int idx_row_len, int nqb_f, int nkb_f, int g, int nqt, int nkt,
+                         int32_t* t_cnt, int32_t* t_idx, uint64_t* t_mask, int32_t* dev_status) {
+  extern __shared__ uint64_t masks[];
+  uint32_t* bits = reinterpret_cast<uint32_t*>(masks + nkt);
+  const int T = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nwords = (nkt + 31) >> 5;
+  for (int i = threadIdx.x; i < nkt; i += blockDim.x) masks[i] = 0ull;
+  __syncthreads();
+  int bad = 0;
+  for (int qi = 0; qi < g; ++qi) {
+    const int qbf = T * g + qi;
+    if (qbf >= nqb_f) break;
+    const int64_t row = b * l_sb + h * l_sh + qbf;
+    int n = kv_cnt[row];
+    if (n < 0 || n > idx_row_len) {
+      bad = 1;
+      n = n < 0 ? 0 : idx_row_len;
+    }
+    const int32_t* list = kv_idx + row * idx_row_len;
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+      const int kb = list[e];
+      if (kb < 0 || kb >= nkb_f) {
+        bad = 1;
+        continue;
+      }
+      atomicOr(reinterpret_cast<unsigned long long*>(&masks[kb / g]),
+               1ull << (qi * g + kb % g));
+    }
+  }
+  if (bad && dev_status) atomicOr(dev_status, 0x1);
+  __syncthreads();
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) {
+    uint32_t word = 0u;
+    for (int i = 0; i < 32; ++i) {
+      const int kt = w * 32 + i;
+      if (kt < nkt && masks[kt] != 0ull) word |= 1u << i;
+    }
+    bits[w] = word;
+  }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int64_t orow = (static_cast<int64_t>(b) * gridDim.y + h) * nqt + T;
+  int32_t* idx_row = t_idx + orow * nkt;
+  uint64_t* mask_row = t_mask + orow * nkt;
+  const int lane = threadIdx.x;
+  int base = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t word = w < nwords ? bits[w] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = base + incl - c;
+    uint32_t rest = word;
+    while (rest) {
+      const int kt = w * 32 + __ffs(rest) - 1;
+      rest &= rest - 1;
+      idx_row[pos] = kt;
+      mask_row[pos] = masks[kt];
+      ++pos;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int i = base + lane; i < nkt; i += 32) {
+    idx_row[i] = -1;
+    mask_row[i] = 0ull;
+  }
+  if (lane == 0) t_cnt[orow] = base;
 }
 
 // ---------------------------------------------------------------- validation

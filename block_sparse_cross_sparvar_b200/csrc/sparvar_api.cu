@@ -241,6 +241,45 @@ int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_idx, int B, i
   return SPARVAR_OK;
 }
 
+int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_idx,
+                          const int64_t* list_strides, int idx_row_len, int B, int H, int Lq,
+                          int Lkv, int block, int32_t* tile_cnt, int32_t* tile_idx,
+                          uint64_t* tile_mask, int32_t* dev_status, void* stream) {
+  if (block != 16 && block != 32 && block != 64)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "block=%d not in {16, 32, 64}", block);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  if (!kv_cnt || !kv_idx || !list_strides || !tile_cnt || !tile_idx || !tile_mask)
+    return fail(SPARVAR_ERR_INVALID_ARG, "a list pointer is NULL");
+  if (list_strides[0] < 0 || list_strides[1] < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
+  if (idx_row_len < 0) return fail(SPARVAR_ERR_INVALID_ARG, "idx_row_len < 0");
+  const int nqt = static_cast<int>(ceil_div(Lq, 128));
+  const int nkt = static_cast<int>(ceil_div(Lkv, 128));
+  if (nkt > 4096)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "Lkv=%d gives %d KV tiles (max 4096)", Lkv, nkt);
+  if (nqt > 65535) return fail(SPARVAR_ERR_UNSUPPORTED, "Lq=%d gives too many query tiles", Lq);
+  const int Bo = list_strides[0] == 0 ? 1 : B;
+  const int Ho = list_strides[1] == 0 ? 1 : H;
+  const int g = 128 / block;
+  const size_t smem = static_cast<size_t>(nkt) * 8 + static_cast<size_t>((nkt + 31) / 32) * 4;
+  cudaError_t e = cudaFuncSetAttribute(sparvar::coarsen_lists_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  dim3 grid(nqt, Ho, Bo);
+  sparvar::coarsen_lists_kernel<<<grid, sparvar::kMaskThreads, smem,
+                                  static_cast<cudaStream_t>(stream)>>>(
+      kv_cnt, kv_idx, list_strides[0], list_strides[1], idx_row_len,
+      static_cast<int>(ceil_div(Lq, block)), static_cast<int>(ceil_div(Lkv, block)), g, nqt, nkt,
+      tile_cnt, tile_idx, tile_mask, dev_status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "coarsen_lists_kernel launch");
+  return SPARVAR_OK;
+}
+
 int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_rows,
                            int idx_row_len, int nkb, int32_t* dev_status, void* stream) {
   if (!kv_cnt || !kv_idx || !dev_status)
@@ -262,7 +301,8 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
                                   const int64_t* q_strides, const int64_t* k_strides,
                                   const int64_t* v_strides, const int64_t* o_strides,
                                   const int32_t* kv_cnt, const int32_t* kv_idx,
-                                  const int64_t* list_strides, int idx_row_len, int block_q,
+                                  const int64_t* list_strides, int idx_row_len,
+                                  const uint64_t* tile_mask, int mask_block, int block_q,
                                   int block_kv, float softmax_scale, int32_t* dev_status,
                                   void* stream) {
   if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
@@ -286,6 +326,12 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   if (list_strides[0] < 0 || list_strides[1] < 0)
     return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
   if (idx_row_len < 0) return fail(SPARVAR_ERR_INVALID_ARG, "idx_row_len < 0");
+  int mask_shift = 7;
+  if (tile_mask) {
+    if (mask_block != 16 && mask_block != 32 && mask_block != 64)
+      return fail(SPARVAR_ERR_UNSUPPORTED, "mask_block=%d not in {16, 32, 64}", mask_block);
+    mask_shift = mask_block == 16 ? 4 : (mask_block == 32 ? 5 : 6);
+  }
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f))
     return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
 
@@ -297,6 +343,8 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   a.kv_cnt = kv_cnt; a.kv_idx = kv_idx;
   a.list_sb = list_strides[0]; a.list_sh = list_strides[1];
   a.idx_row_len = idx_row_len;
+  a.tile_mask = tile_mask;
+  a.mask_shift = mask_shift;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
   a.lse = lse;

@@ -37,8 +37,10 @@ EXPORTS = {
     "sparvar_map_indices": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
                              _vp], _i),
     "sparvar_block_sparse_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p,
-                                       _i64p, _i64p, _vp, _vp, _i64p, _i, _i, _i, _f, _vp, _vp],
-                                      _i),
+                                       _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _i, _i, _i, _f, _vp,
+                                       _vp], _i),
+    "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
+                              _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
 }
 
@@ -133,9 +135,37 @@ def _list_strides(kv_cnt, B, H):
     raise SparvarError("kv_cnt must be 1-, 2- or 3-D")
 
 
+def sparvar_coarsen_lists(kv_cnt, kv_idx, B, H, Lq, Lkv, block, dev_status=None):
+    """Fine (16/32/64) block lists -> 128x128 tile lists and per-tile masks.
+
+    Returns (tile_cnt [Bo, Ho, NQT], tile_idx [Bo, Ho, NQT, NKT], tile_mask, same
+    shape, int64 holding the uint64 bits), Bo/Ho = 1 where the input lists are
+    shared across batch items/heads."""
+    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32:
+        raise SparvarError("kv_cnt/kv_idx must be int32")
+    if kv_idx.shape[:-1] != kv_cnt.shape or not kv_idx.is_contiguous():
+        raise SparvarError("kv_idx must be contiguous with shape (*kv_cnt.shape, row_len)")
+    if kv_cnt.shape[-1] != -(-Lq // block):
+        raise SparvarError(f"kv_cnt has {kv_cnt.shape[-1]} query blocks, expected {-(-Lq // block)}")
+    sb, sh = _list_strides(kv_cnt, B, H)
+    Bo, Ho = (1 if sb == 0 else B), (1 if sh == 0 else H)
+    nqt, nkt = -(-Lq // 128), -(-Lkv // 128)
+    dev = kv_cnt.device
+    t_cnt = torch.empty(Bo, Ho, nqt, dtype=torch.int32, device=dev)
+    t_idx = torch.empty(Bo, Ho, nqt, nkt, dtype=torch.int32, device=dev)
+    t_mask = torch.empty(Bo, Ho, nqt, nkt, dtype=torch.int64, device=dev)
+    _check(lib().sparvar_coarsen_lists(_ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1],
+                                       B, H, Lq, Lkv, block, _ptr(t_cnt), _ptr(t_idx), _ptr(t_mask),
+                                       _ptr(dev_status), _stream(dev)), "sparvar_coarsen_lists")
+    return t_cnt, t_idx, t_mask
+
+
 def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv=128,
                                   softmax_scale=None, out=None, return_lse=False, dev_status=None):
-    """Block-sparse attention forward: returns O (and the row LSE when asked)."""
+    """Block-sparse attention forward: returns O (and the row LSE when asked).
+
+    Lists over 128x128 blocks go to the kernel as they are; lists over square
+    16/32/64 blocks are first coarsened to 128x128 tiles with per-tile masks."""
     B, H, Lq, D = q.shape
     Lkv = k.shape[2]
     if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
@@ -151,13 +181,20 @@ def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv
     nqb = -(-Lq // block_q)
     if kv_cnt.shape[-1] != nqb:
         raise SparvarError(f"kv_cnt has {kv_cnt.shape[-1]} query blocks, expected {nqb}")
+    tile_mask, mask_block = None, 0
+    if (block_q, block_kv) != (128, 128):
+        if block_q != block_kv or block_q not in (16, 32, 64):
+            raise SparvarError(f"blocks ({block_q}, {block_kv}): 128 x 128 or square 16/32/64")
+        kv_cnt, kv_idx, tile_mask = sparvar_coarsen_lists(kv_cnt, kv_idx, B, H, Lq, Lkv, block_q,
+                                                          dev_status)
+        mask_block = block_q
     lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     sb, sh = _list_strides(kv_cnt, B, H)
     _check(lib().sparvar_block_sparse_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
-        _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], block_q, block_kv, scale,
-        _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd")
+        _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], _ptr(tile_mask), mask_block,
+        128, 128, scale, _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd")
     return (out, lse) if return_lse else out
 
 

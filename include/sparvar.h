@@ -177,7 +177,15 @@ SPARVAR_API int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_i
  *            kv_idx[(b*list_strides[0] + h*list_strides[1] + qb) * idx_row_len].
  *            list_strides (host, 2 values, in list rows) may be 0 to share one
  *            list set across batch items or heads.
- * block_q = block_kv = 128.
+ * tile_mask  device uint64 or NULL.  NULL: the lists name whole 128x128 blocks.
+ *            Otherwise the lists name 128x128 tiles of a finer square block grid
+ *            of side mask_block (16, 32 or 64; g = 128 / mask_block), as written
+ *            by sparvar_coarsen_lists: entry e of list row r has its mask at
+ *            tile_mask[r * idx_row_len + e], and bit (qi * g + ki) keeps fine KV
+ *            block ki of the tile for the tile's fine query block qi.  Keys of a
+ *            fine block whose bit is clear are excluded for that block's rows.
+ * mask_block ignored when tile_mask is NULL.
+ * block_q = block_kv = 128 (the tile size of the lists).
  * dev_status device int32 or NULL: SPARVAR_DEV_BAD_LIST when an entry is out of
  *            range (the entry contributes nothing), SPARVAR_DEV_TIMEOUT when a
  *            bounded wait gave up.
@@ -187,9 +195,37 @@ SPARVAR_API int sparvar_block_sparse_attn_fwd(const void* q, const void* k, cons
                                   const int64_t* q_strides, const int64_t* k_strides,
                                   const int64_t* v_strides, const int64_t* o_strides,
                                   const int32_t* kv_cnt, const int32_t* kv_idx,
-                                  const int64_t* list_strides, int idx_row_len, int block_q,
+                                  const int64_t* list_strides, int idx_row_len,
+                                  const uint64_t* tile_mask, int mask_block, int block_q,
                                   int block_kv, float softmax_scale, int32_t* dev_status,
                                   void* stream);
+
+/*
+ * Fine block lists to 128x128 tile lists with per-tile bitmasks, the form the
+ * attention call takes for block sizes below 128 ("Main Findings" block-size
+ * rows: the mask is defined on a fine grid, the contraction runs on 128x128
+ * tensor-core tiles).
+ *
+ * Input: lists over square blocks of side `block` (16, 32 or 64) for queries
+ *   [0, Lq) and keys [0, Lkv): count of (b, h, fine query block qb) at
+ *   kv_cnt[b*list_strides[0] + h*list_strides[1] + qb], entries (fine KV block
+ *   indices) from kv_idx[(that row) * idx_row_len]; list_strides (host, 2 values)
+ *   may be 0 to share lists.
+ * Output, for Bo = (list_strides[0] == 0 ? 1 : B) and Ho = (list_strides[1] == 0
+ *   ? 1 : H), NQT = ceil(Lq/128), NKT = ceil(Lkv/128) (NKT <= 4096):
+ *   tile_cnt int32 [Bo][Ho][NQT], tile_idx int32 [Bo][Ho][NQT][NKT] (ascending,
+ *   -1 padded), tile_mask uint64 [Bo][Ho][NQT][NKT] (0 padded), all device,
+ *   caller-allocated.  Pass them to sparvar_block_sparse_attn_fwd with
+ *   list_strides {Bo > 1 ? Ho*NQT : 0, Ho > 1 ? NQT : 0}, idx_row_len NKT and
+ *   mask_block = block.
+ * dev_status device int32 or NULL: SPARVAR_DEV_BAD_LIST for counts or entries out
+ *   of range (skipped).  Duplicated entries are harmless.
+ */
+SPARVAR_API int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_idx,
+                                      const int64_t* list_strides, int idx_row_len, int B, int H,
+                                      int Lq, int Lkv, int block, int32_t* tile_cnt,
+                                      int32_t* tile_idx, uint64_t* tile_mask,
+                                      int32_t* dev_status, void* stream);
 
 /*
  * Device-side check of block lists: for each of n_rows rows,

@@ -120,6 +120,96 @@ def test_attention_tiny_schedule_block128(D):
     _check_attention(q_bits, d["k"][:, :, kv], d["v"][:, :, kv], (cnt, idx), 128, 128, D)
 
 
+@pytest.mark.parametrize("q_scale", [2, 3, 4])
+def test_attention_tiny_schedule_block16(q_scale):
+    """The tiny schedule with 16x16 CSLA blocks (sink = scales 1-2, radius 1), B1 H2
+    D64: fine lists go through coarsening to 128x128 tiles with per-tile masks."""
+    d = inputs.make_qkv(6, 1, 2, TINY, 64, 2, pe=False)
+    off = d["offsets"]
+    q_bits = d["q"][:, :, off[q_scale]:off[q_scale + 1]]
+    kv = slice(0, off[q_scale + 1])
+    cnt, idx, _ = ops.sparvar_build_csla_mask(TINY, q_scale, 2, 1, 1, 16, 16)
+    _check_attention(q_bits, d["k"][:, :, kv], d["v"][:, :, kv], (cnt, idx), 16, 16, 64)
+
+
+def _random_lists(rng, B, H, nqb, nkb, p):
+    blk = rng.random((B, H, nqb, nkb)) < p
+    cnt = torch.from_numpy(blk.sum(-1).astype(np.int32)).cuda()
+    idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                kept = np.nonzero(blk[b, h, qb])[0]
+                idx_np[b, h, qb, :kept.size] = kept
+    return blk, cnt, torch.from_numpy(idx_np).cuda()
+
+
+@pytest.mark.parametrize("block,D", [(16, 64), (32, 128), (64, 128), (16, 128)])
+def test_attention_fine_blocks_random_lists(block, D):
+    """Random per-(b, h) fine lists with ragged query and key tails, an empty row
+    and a row whose only blocks sit in the ragged last tile."""
+    rng = np.random.default_rng(block + D)
+    B, H, Lq, Lkv = 2, 2, 300, 777
+    bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
+            for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
+    nqb, nkb = -(-Lq // block), -(-Lkv // block)
+    blk, cnt, idx = _random_lists(rng, B, H, nqb, nkb, 0.3)
+    cnt[0, 0, 1] = 0
+    cnt[1, 1, nqb - 1] = 1
+    idx[1, 1, nqb - 1, 0] = nkb - 1
+    _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), block, block, D, scale=0.1)
+
+
+@pytest.mark.parametrize("block", [16, 32, 64])
+def test_coarsen_lists_bit_exact(block):
+    """Tile lists and masks expand to exactly the fine block mask."""
+    rng = np.random.default_rng(7 * block)
+    B, H, Lq, Lkv = 2, 3, 1000, 2100
+    nqb, nkb = -(-Lq // block), -(-Lkv // block)
+    blk, cnt, idx = _random_lists(rng, B, H, nqb, nkb, 0.2)
+    st = _status()
+    t_cnt, t_idx, t_mask = ops.sparvar_coarsen_lists(cnt, idx, B, H, Lq, Lkv, block, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    t_cnt, t_idx = t_cnt.cpu().numpy(), t_idx.cpu().numpy()
+    t_mask = t_mask.cpu().numpy().view(np.uint64)
+    g, nqt, nkt = 128 // block, -(-Lq // 128), -(-Lkv // 128)
+    for b in range(B):
+        for h in range(H):
+            got = np.zeros((nqt * g, nkt * g), bool)
+            for T in range(nqt):
+                c = t_cnt[b, h, T]
+                row = t_idx[b, h, T]
+                assert np.all(np.diff(row[:c]) > 0) and np.all(row[c:] == -1)
+                assert np.all(t_mask[b, h, T, c:] == 0)
+                for e in range(c):
+                    m = int(t_mask[b, h, T, e])
+                    assert m != 0
+                    for qi in range(g):
+                        for ki in range(g):
+                            if (m >> (qi * g + ki)) & 1:
+                                got[T * g + qi, row[e] * g + ki] = True
+            assert np.array_equal(got[:nqb, :nkb], blk[b, h])
+            assert not got[nqb:].any() and not got[:, nkb:].any()
+
+
+def test_coarsen_shared_lists_stay_shared():
+    cnt, idx, blk = ops.sparvar_build_csla_mask(TINY, 4, 2, 1, 1, 16, 16, with_mask=True)
+    t_cnt, t_idx, t_mask = ops.sparvar_coarsen_lists(cnt, idx, 2, 4, 256, 341, 16)
+    assert tuple(t_cnt.shape) == (1, 1, 2) and tuple(t_idx.shape) == (1, 1, 2, 3)
+    ocnt, oidx, oblk = orc.build_csla_mask(TINY, 4, 2, 1, 1, 16, 16)
+    m = t_mask.cpu().numpy().view(np.uint64)[0, 0]
+    ti = t_idx.cpu().numpy()[0, 0]
+    for T in range(2):
+        for e in range(int(t_cnt[0, 0, T])):
+            for qi in range(8):
+                for ki in range(8):
+                    qb, kb = T * 8 + qi, ti[T, e] * 8 + ki
+                    bit = bool((int(m[T, e]) >> (qi * 8 + ki)) & 1)
+                    exp = qb < oblk.shape[0] and kb < oblk.shape[1] and bool(oblk[qb, kb])
+                    assert bit == exp
+
+
 @pytest.mark.parametrize("q_scale,D", [(9, 128), (10, 128), (10, 64), (8, 128)])
 def test_attention_infinity_mid_scales(q_scale, D):
     d = inputs.make_qkv(2, 1, 2, INF, D, 5)

@@ -45,14 +45,15 @@ def _attn_call(lib, **over):
     i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
     args = dict(q=16, k=16, v=16, o=16, lse=0, B=1, H=1, Lq=128, Lkv=128, D=128,
                 qs=i64(0, 0, 128), ks=i64(0, 0, 128), vs=i64(0, 0, 128), os=i64(0, 0, 128),
-                cnt=16, idx=16, ls=i64(0, 0), row=1, bq=128, bk=128, scale=0.1, st=0, stream=0)
+                cnt=16, idx=16, ls=i64(0, 0), row=1, tm=0, mb=0, bq=128, bk=128, scale=0.1, st=0,
+                stream=0)
     args.update(over)
     vp = ctypes.c_void_p
     return lib.sparvar_block_sparse_attn_fwd(
         vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["o"]), vp(args["lse"]), args["B"],
         args["H"], args["Lq"], args["Lkv"], args["D"], args["qs"], args["ks"], args["vs"], args["os"],
-        vp(args["cnt"]), vp(args["idx"]), args["ls"], args["row"], args["bq"], args["bk"],
-        args["scale"], vp(args["st"]), vp(args["stream"]))
+        vp(args["cnt"]), vp(args["idx"]), args["ls"], args["row"], vp(args["tm"]), args["mb"],
+        args["bq"], args["bk"], args["scale"], vp(args["st"]), vp(args["stream"]))
 
 
 @pytest.mark.parametrize("over,code,msg", [
@@ -64,6 +65,8 @@ def _attn_call(lib, **over):
     (dict(cnt=0), 1, "kv_cnt"),
     (dict(row=-1), 1, "idx_row_len"),
     (dict(scale=float("inf")), 1, "softmax_scale"),
+    (dict(tm=16, mb=8), 2, "mask_block=8"),
+    (dict(tm=16, mb=128), 2, "mask_block=128"),
 ])
 def test_attention_rejects_bad_arguments_on_host(lib, over, code, msg):
     assert _attn_call(lib, **over) == code
@@ -101,3 +104,20 @@ def test_map_and_decide_reject_bad_arguments(lib):
                                      vp(0), vp(0), vp(0)) == 2
     assert "KV blocks" in lib.sparvar_last_error().decode()
     assert lib.sparvar_validate_lists(vp(16), vp(16), 4, 4, 4, vp(0), vp(0)) == 1
+
+
+def test_coarsen_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+
+    def call(block=16, B=1, H=1, Lq=256, Lkv=256, cnt=16, ls=None, row=16, lkv_ok=True):
+        return lib.sparvar_coarsen_lists(vp(cnt), vp(16), ls if ls is not None else i64(0, 0), row,
+                                         B, H, Lq, Lkv, block, vp(16), vp(16), vp(16), vp(0), vp(0))
+
+    assert call(block=128) == 2 and "block=128" in lib.sparvar_last_error().decode()
+    assert call(block=8) == 2
+    assert call(cnt=0) == 1 and "NULL" in lib.sparvar_last_error().decode()
+    assert call(Lq=0) == 1
+    assert call(ls=i64(-1, 0)) == 1
+    assert call(row=-1) == 1
+    assert call(Lkv=4097 * 128) == 2 and "KV tiles" in lib.sparvar_last_error().decode()
