@@ -264,10 +264,49 @@ def select_blocks_by_mass(M, mass_threshold):
     return blk, margin
 
 
-def decide_blocks(q, k, block_q, block_kv, mass_threshold, scale=None):
-    """Decision-scale block selection for one (batch, head): (cnt, idx, blk, M, margin)."""
+def topk_count(ratio, nkb):
+    """Blocks kept per query block in the Top-K mode.
+
+    [M] CS4A uses "a Top-K operation to find which keys matter most", with
+    "Top-K around 0.2" as the pages' default; read as a ratio of the key blocks:
+    k = ceil(ratio * NKB), at least 1 and at most NKB.  The product is taken with
+    a 1e-6 allowance so that a ratio given in binary floating point (0.2 is
+    0.2000000030 as a float32) does not round 0.2 * 20 up to 5.
+    """
+    return int(min(nkb, max(1, math.ceil(ratio * nkb - 1e-6))))
+
+
+def select_blocks_topk(M, ratio):
+    """Per query block keep the topk_count(ratio, NKB) blocks of largest mass.
+
+    Ties are broken towards the smaller block index.  Returns (blk, margin) with
+    margin [NQB] the mass gap between the last kept and the first dropped block
+    (inf when every block is kept): the decision flips only if masses move by
+    more than that.
+    """
+    nqb, nkb = M.shape
+    k = topk_count(ratio, nkb)
+    blk = np.zeros((nqb, nkb), dtype=bool)
+    margin = np.full(nqb, np.inf)
+    for qb in range(nqb):
+        order = sorted(range(nkb), key=lambda kb: (-M[qb, kb], kb))
+        for kb in order[:k]:
+            blk[qb, kb] = True
+        if k < nkb:
+            margin[qb] = M[qb, order[k - 1]] - M[qb, order[k]]
+    return blk, margin
+
+
+def decide_blocks(q, k, block_q, block_kv, mass_threshold, scale=None, topk_ratio=None):
+    """Decision-scale block selection for one (batch, head): (cnt, idx, blk, M, margin).
+
+    The mass-threshold rule by default; the Top-K-ratio rule when ``topk_ratio``
+    is given."""
     M = decision_block_mass(q, k, block_q, block_kv, scale)
-    blk, margin = select_blocks_by_mass(M, mass_threshold)
+    if topk_ratio is not None:
+        blk, margin = select_blocks_topk(M, topk_ratio)
+    else:
+        blk, margin = select_blocks_by_mass(M, mass_threshold)
     cnt, idx = block_lists(blk)
     return cnt, idx, blk, M, margin
 

@@ -110,6 +110,47 @@ def test_select_golden():
         assert list(np.nonzero(blk[0])[0]) == want, line
 
 
+def test_select_topk_golden():
+    for line in open(os.path.join(GOLDEN, "select_topk.txt")):
+        if not line.startswith("ratio"):
+            continue
+        a, b, c = line.split("|")
+        ratio = float(a.split()[1])
+        M = np.array([[float(x) for x in b.split()]])
+        want = [int(x) for x in c.split()]
+        blk, margin = orc.select_blocks_topk(M, ratio)
+        assert list(np.nonzero(blk[0])[0]) == want, line
+
+
+@pytest.mark.parametrize("ratio,nkb,k", [(0.2, 20, 4), (np.float32(0.2), 20, 4), (0.2, 83, 17),
+                                         (0.2, 51, 11), (0.2, 5, 1), (0.2, 1, 1), (1e-9, 40, 1),
+                                         (1.0, 33, 33), (0.5, 7, 4), (0.25, 8, 2)])
+def test_topk_count(ratio, nkb, k):
+    assert orc.topk_count(float(ratio), nkb) == k
+
+
+def test_topk_special_cases_and_order():
+    q, k = _rand(6, 64, 16), _rand(7, 100, 16)
+    M = orc.decision_block_mass(q, k, 16, 16)
+    blk1, _ = orc.select_blocks_topk(M, 1e-9)
+    assert np.array_equal(np.nonzero(blk1)[1], np.argmax(M, axis=1))
+    blk_all, margin = orc.select_blocks_topk(M, 1.0)
+    assert blk_all.all() and np.isinf(margin).all()
+    blk, margin = orc.select_blocks_topk(M, 0.3)
+    kk = orc.topk_count(0.3, M.shape[1])
+    for qb in range(M.shape[0]):
+        assert blk[qb].sum() == kk
+        # every kept block is at least as heavy as every dropped one, by the margin
+        assert M[qb][blk[qb]].min() - M[qb][~blk[qb]].max() == pytest.approx(margin[qb])
+        assert margin[qb] >= 0
+    # the mass rule's set for a row is the Top-K set with k = its size
+    blk_m, _ = orc.select_blocks_by_mass(M, 0.8)
+    for qb in range(M.shape[0]):
+        n = int(blk_m[qb].sum())
+        bk, _ = orc.select_blocks_topk(M[qb:qb + 1], (n - 0.5) / M.shape[1])
+        assert np.array_equal(bk[0], blk_m[qb])
+
+
 def _rand(seed, *shape):
     return np.random.default_rng(seed).standard_normal(shape)
 
