@@ -56,6 +56,7 @@ struct AttnArgs {
   // mass mode
   const float* lse_in;  // [B][H][Lq] natural log, or null -> computed in a first sweep
   float mass_threshold;
+  int topk;          // > 0: keep exactly this many blocks per query block (Top-K mode)
   int32_t* sel_cnt;  // [B][H][nqb]
   int32_t* sel_idx;  // [B][H][nqb][nkb]
   float* mass_out;   // [B][H][nqb][nkb] or null
@@ -466,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         float run = 0.f;
         int taken = 0;
-        while (taken < nkb) {
+        const int limit = args.topk > 0 ? min(args.topk, nkb) : nkb;
+        while (taken < limit) {
           float best = -1.f;
           int best_i = 0x7fffffff;
           for (int i = lane; i < nkb; i += 32) {
@@ -485,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           run += best;
           ++taken;
-          if (run >= args.mass_threshold) break;
+          if (args.topk <= 0 && run >= args.mass_threshold) break;
         }
         // ascending compaction
         int base = 0;

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -363,8 +364,8 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
 int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
                           const int64_t* q_strides, const int64_t* k_strides, float softmax_scale,
                           const float* lse, int block_q, int block_kv, float mass_threshold,
-                          int32_t* kv_cnt, int32_t* kv_idx, float* mass, int32_t* dev_status,
-                          void* stream) {
+                          float topk_ratio, int32_t* kv_cnt, int32_t* kv_idx, float* mass,
+                          int32_t* dev_status, void* stream) {
   if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
   if (block_q != 128 || block_kv != 128)
     return fail(SPARVAR_ERR_UNSUPPORTED, "decision blocks (%d, %d): 128 x 128 only", block_q,
@@ -383,6 +384,8 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   if (!kv_cnt || !kv_idx) return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx is NULL");
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f) || std::isnan(mass_threshold))
     return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0, mass_threshold a number");
+  if (!(topk_ratio >= 0.f && topk_ratio <= 1.f))
+    return fail(SPARVAR_ERR_INVALID_ARG, "topk_ratio must be in [0, 1] (0: mass threshold)");
 
   sparvar::AttnArgs a{};
   a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
@@ -391,6 +394,11 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.lse_in = lse;
   a.mass_threshold = mass_threshold;
+  // k = ceil(ratio * NKB), at least one; the allowance keeps 0.2f * 20 at 4
+  a.topk = topk_ratio > 0.f
+               ? static_cast<int>(std::min<double>(
+                     nkb, std::max<double>(1.0, std::ceil(static_cast<double>(topk_ratio) * nkb - 1e-6))))
+               : 0;
   a.sel_cnt = kv_cnt; a.sel_idx = kv_idx; a.mass_out = mass;
   a.dev_status = dev_status;
   CUtensorMap tq, tk;

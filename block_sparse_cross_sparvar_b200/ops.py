@@ -33,7 +33,7 @@ EXPORTS = {
     "sparvar_scale_blocks": ([_i32p, _i, _i, _i, _i, _i32p, _i32p], _i),
     "sparvar_build_csla_mask": ([_i32p, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "sparvar_decide_blocks": ([_vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p, _f, _vp, _i, _i, _f,
-                               _vp, _vp, _vp, _vp, _vp], _i),
+                               _f, _vp, _vp, _vp, _vp, _vp], _i),
     "sparvar_map_indices": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
                              _vp], _i),
     "sparvar_block_sparse_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p,
@@ -199,8 +199,10 @@ def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv
 
 
 def sparvar_decide_blocks(q, k, mass_threshold, lse=None, softmax_scale=None, block_q=128,
-                          block_kv=128, return_mass=False, dev_status=None):
-    """CS4A decision: (kv_cnt [B,H,NQB], kv_idx [B,H,NQB,NKB], mass|None)."""
+                          block_kv=128, return_mass=False, dev_status=None, topk_ratio=0.0):
+    """CS4A decision: (kv_cnt [B,H,NQB], kv_idx [B,H,NQB,NKB], mass|None).
+
+    mass_threshold rule by default; topk_ratio > 0 keeps ceil(ratio * NKB) blocks."""
     B, H, Lq, D = q.shape
     Lkv = k.shape[2]
     qs, ks = _bhrd(q, "q"), _bhrd(k, "k")
@@ -214,7 +216,8 @@ def sparvar_decide_blocks(q, k, mass_threshold, lse=None, softmax_scale=None, bl
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     _check(lib().sparvar_decide_blocks(
         _ptr(q), _ptr(k), B, H, Lq, Lkv, D, qs, ks, scale, _ptr(lse), block_q, block_kv,
-        float(mass_threshold), _ptr(cnt), _ptr(idx), _ptr(mass), _ptr(dev_status),
+        float(mass_threshold), float(topk_ratio), _ptr(cnt), _ptr(idx), _ptr(mass),
+        _ptr(dev_status),
         _stream(q.device)), "sparvar_decide_blocks")
     return cnt, idx, mass
 

@@ -115,8 +115,11 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
  *   s = softmax_scale * q . key over all Lkv keys (no mask), lse = log-sum-exp of row q.
  * Per query block, KV blocks are ordered by mass (descending, ties to the lower
  * index) and the shortest prefix whose running sum reaches mass_threshold is
- * kept (every block when the total stays below it).  Kept lists are written in
- * ascending order.
+ * kept (every block when the total stays below it).  With topk_ratio > 0 the
+ * first k = ceil(topk_ratio * nkb) blocks of that order are kept instead (at
+ * least one; the product is taken with a 1e-6 allowance so 0.2 * 20 gives 4):
+ * the Top-K rule of the same paragraph, "Top-K around 0.2" in "Main Findings".
+ * Kept lists are written in ascending order.
  *
  * q [B][H][Lq][D], k [B][H][Lkv][D]: device bf16; strides in elements for
  *   (b, h, row) given by host arrays q_strides[3], k_strides[3]; row strides and
@@ -124,6 +127,7 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
  * lse        device fp32 [B][H][Lq] contiguous (natural log), or NULL to have the
  *            call compute it (one extra sweep over the keys).
  * block_q = block_kv = 128.
+ * mass_threshold  used when topk_ratio == 0.  topk_ratio in [0, 1].
  * kv_cnt     device int32 [B][H][nqb]; kv_idx device int32 [B][H][nqb][nkb] (-1 padded).
  * mass       device fp32 [B][H][nqb][nkb] or NULL.
  * dev_status device int32 or NULL.
@@ -131,8 +135,8 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
 SPARVAR_API int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,
                           const int64_t* q_strides, const int64_t* k_strides,
                           float softmax_scale, const float* lse, int block_q, int block_kv,
-                          float mass_threshold, int32_t* kv_cnt, int32_t* kv_idx, float* mass,
-                          int32_t* dev_status, void* stream);
+                          float mass_threshold, float topk_ratio, int32_t* kv_cnt,
+                          int32_t* kv_idx, float* mass, int32_t* dev_status, void* stream);
 
 /*
  * CS4A cross-scale index mapping ("Methodology in Plain English", CS4A

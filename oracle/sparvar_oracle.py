@@ -362,6 +362,83 @@ def map_indices(src_cnt, src_idx, src_nq, src_lkv, dst_nq, dst_lkv, block_q, blo
     return cnt, idx, dst
 
 
+def upscale_cell(i, s_src, s_dst):
+    """Rows (or columns) [floor(i*s_dst/s_src), ceil((i+1)*s_dst/s_src)) of a
+    side-s_dst grid covered by row (column) i of a side-s_src grid."""
+    return (i * s_dst) // s_src, -((-(i + 1) * s_dst) // s_src)
+
+
+def map_block_mask_2d(src_blk, sides, src_scale, dst_scale, block_q, block_kv, n_sink_tokens):
+    """Scale-aware 2-D reading of the CS4A mapping (the alternative to
+    ``map_block_mask``).
+
+    [M] CS4A maps the selected indices "to later, larger scales by rescaling the
+    index positions" and calls the result scale self-similar.  Reading: a query
+    token (i, j) of the decision scale (side s_d) stands for its upscaled cell of
+    the target scale (side s_t): rows upscale_cell(i), columns upscale_cell(j).  A
+    key keeps its position when it lies in a scale before the decision scale (the
+    target's prefix holds the same tokens), and a key of the decision scale
+    itself at (a, b) stands for the cell of (a, b) in the target scale's own
+    tokens.  Keys of the scales between the two are reached only through the
+    sink.  Every destination (query block, KV block) pair holding a mapped query
+    and a mapped key of one kept source pair is kept; the union is taken over
+    kept source pairs, and every KV block holding a key below ``n_sink_tokens``
+    is added to every row.
+    """
+    off = scale_offsets(sides)
+    s_d, s_t = sides[src_scale], sides[dst_scale]
+    n_d, n_t = s_d * s_d, s_t * s_t
+    l_d, l_t = off[src_scale + 1], off[dst_scale + 1]
+    d_nqb, d_nkb = n_blocks(n_t, block_q), n_blocks(l_t, block_kv)
+    dst = np.zeros((d_nqb, d_nkb), dtype=bool)
+
+    def query_blocks(qb):
+        out = set()
+        for q in range(qb * block_q, min((qb + 1) * block_q, n_d)):
+            i, j = divmod(q, s_d)
+            r0, r1 = upscale_cell(i, s_d, s_t)
+            c0, c1 = upscale_cell(j, s_d, s_t)
+            for r in range(r0, r1):
+                for c in range(c0, c1):
+                    out.add((r * s_t + c) // block_q)
+        return out
+
+    def key_blocks(kb):
+        out = set()
+        for key in range(kb * block_kv, min((kb + 1) * block_kv, l_d)):
+            if key < off[src_scale]:
+                out.add(key // block_kv)
+                continue
+            a, b = divmod(key - off[src_scale], s_d)
+            r0, r1 = upscale_cell(a, s_d, s_t)
+            c0, c1 = upscale_cell(b, s_d, s_t)
+            for r in range(r0, r1):
+                for c in range(c0, c1):
+                    out.add((off[dst_scale] + r * s_t + c) // block_kv)
+        return out
+
+    qsets = [query_blocks(qb) for qb in range(src_blk.shape[0])]
+    ksets = [key_blocks(kb) for kb in range(src_blk.shape[1])]
+    for qb, kb in zip(*np.nonzero(src_blk)):
+        for tq in qsets[qb]:
+            for tk in ksets[kb]:
+                dst[tq, tk] = True
+    if n_sink_tokens > 0:
+        dst[:, :n_blocks(min(n_sink_tokens, l_t), block_kv)] = True
+    return dst
+
+
+def map_indices_2d(src_cnt, src_idx, sides, src_scale, dst_scale, block_q, block_kv,
+                   n_sink_tokens):
+    """List form of ``map_block_mask_2d``: (cnt, idx, blk) on the destination grid."""
+    off = scale_offsets(sides)
+    src_blk = lists_to_blocks(src_cnt, src_idx, n_blocks(off[src_scale + 1], block_kv))
+    dst = map_block_mask_2d(src_blk, sides, src_scale, dst_scale, block_q, block_kv,
+                            n_sink_tokens)
+    cnt, idx = block_lists(dst)
+    return cnt, idx, dst
+
+
 # ----------------------------------------------------------------------------
 # FLOP accounting for the kept blocks (metric definition)
 # ----------------------------------------------------------------------------

@@ -362,6 +362,40 @@ def test_decide_blocks_with_lse_from_attention():
     _decide_compare(d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]], 0.95, lse_dev=lse)
 
 
+@pytest.mark.parametrize("ratio,D", [(0.2, 128), (0.5, 64), (1e-6, 128), (1.0, 128)])
+def test_decide_blocks_topk_ratio(ratio, D):
+    """Top-K-ratio mode: exactly ceil(ratio * NKB) blocks, the heaviest ones; bit-exact
+    where the gap between the last kept and first dropped mass exceeds 1e-4."""
+    d = inputs.make_qkv(8, 1, 3, INF, D, 5)
+    off = d["offsets"]
+    s = 9
+    q_bits, k_bits = d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]]
+    B, H = q_bits.shape[:2]
+    st = _status()
+    cnt, idx, mass = ops.sparvar_decide_blocks(_dev(q_bits), _dev(k_bits), 0.95, topk_ratio=ratio,
+                                               return_mass=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    cnt, idx, mass = cnt.cpu().numpy(), idx.cpu().numpy(), mass.cpu().numpy()
+    nkb = mass.shape[-1]
+    kk = orc.topk_count(ratio, nkb)
+    assert np.all(cnt == kk)
+    for b in range(B):
+        for h in range(H):
+            ocnt, oidx, oblk, M, margin = orc.decide_blocks(
+                q_bits_f(q_bits, b, h), q_bits_f(k_bits, b, h), 128, 128, None, topk_ratio=ratio)
+            assert np.abs(mass[b, h] - M).max() < 2e-5
+            for qb in range(M.shape[0]):
+                kept = idx[b, h, qb, :kk]
+                assert np.all(np.diff(kept) > 0) and np.all(idx[b, h, qb, kk:] == -1)
+                if margin[qb] > 1e-4:
+                    assert np.array_equal(kept, oidx[qb, :kk])
+                else:  # a valid Top-K set of the kernel's own masses
+                    mk = mass[b, h, qb]
+                    drop = np.setdiff1d(np.arange(nkb), kept)
+                    assert drop.size == 0 or mk[kept].min() >= mk[drop].max()
+
+
 @pytest.mark.parametrize("tau", [0.5, 0.99, 2.0])
 def test_decide_blocks_thresholds_d64(tau):
     d = inputs.make_qkv(2, 1, 2, INF, 64, 5)

@@ -100,9 +100,14 @@ def test_map_and_decide_reject_bad_arguments(lib):
                                    vp(0), vp(0), vp(0)) == 1
     i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
     assert lib.sparvar_decide_blocks(vp(16), vp(16), 1, 1, 128, 600000, 128, i64(0, 0, 128),
-                                     i64(0, 0, 128), 0.1, vp(0), 128, 128, 0.95, vp(16), vp(16),
-                                     vp(0), vp(0), vp(0)) == 2
+                                     i64(0, 0, 128), 0.1, vp(0), 128, 128, 0.95, 0.0, vp(16),
+                                     vp(16), vp(0), vp(0), vp(0)) == 2
     assert "KV blocks" in lib.sparvar_last_error().decode()
+    for bad in (1.5, -0.1, float("nan")):
+        assert lib.sparvar_decide_blocks(vp(16), vp(16), 1, 1, 128, 1000, 128, i64(0, 0, 128),
+                                         i64(0, 0, 128), 0.1, vp(0), 128, 128, 0.95, bad, vp(16),
+                                         vp(16), vp(0), vp(0), vp(0)) == 1
+        assert "topk_ratio" in lib.sparvar_last_error().decode()
     assert lib.sparvar_validate_lists(vp(16), vp(16), 4, 4, 4, vp(0), vp(0)) == 1
 
 

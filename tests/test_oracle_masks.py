@@ -13,6 +13,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
+from block_sparse_cross_sparvar_b200 import inputs
 from oracle import sparvar_oracle as orc
 from tests.conftest import GOLDEN
 
@@ -291,3 +292,99 @@ def test_map_identity_and_invariants():
     for qb in range(32):
         row = idx[qb, :cnt[qb]]
         assert np.all(np.diff(row) > 0)
+
+
+# ---------------------------------------------------------------- CS4A 2-D mapping
+def test_map_2d_golden():
+    for line in open(os.path.join(GOLDEN, "map_2d_tiny.txt")):
+        if not line.startswith("case"):
+            continue
+        parts = [p.strip() for p in line.split("|")]
+        sink = int(parts[1].split()[1])
+        src = np.zeros((2, 3), bool)
+        for pr in parts[2].split():
+            a, b = pr.split(":")
+            src[int(a), int(b)] = True
+        want = np.zeros((8, 11), bool)
+        for pr in parts[3].split():
+            a, b = pr.split(":")
+            for x in filter(None, b.split(",")):
+                want[int(a), int(x)] = True
+        dst = orc.map_block_mask_2d(src, (1, 2, 4), 1, 2, 2, 2, sink)
+        assert np.array_equal(dst, want), parts[0]
+
+
+def test_upscale_cell():
+    assert orc.upscale_cell(3, 4, 8) == (6, 8)          # exact 2x
+    assert orc.upscale_cell(0, 32, 40) == (0, 2)        # 1.25x: [0, 1.25) -> rows 0, 1
+    assert orc.upscale_cell(3, 32, 40) == (3, 5)        # [3.75, 5)
+    assert orc.upscale_cell(31, 32, 48) == (46, 48)
+    assert orc.upscale_cell(5, 7, 7) == (5, 6)          # same side: identity
+
+
+def _token_level_2d(src, sides, d, t, bq, bk, n_sink):
+    """Brute force: token pairs of kept source blocks carried to the target, then blocks."""
+    off = orc.scale_offsets(sides)
+    s_d, s_t = sides[d], sides[t]
+    n_t, l_t = s_t * s_t, off[t + 1]
+    tok = np.zeros((n_t, l_t), bool)
+
+    def img_q(q):
+        i, j = divmod(q, s_d)
+        r0, r1 = orc.upscale_cell(i, s_d, s_t)
+        c0, c1 = orc.upscale_cell(j, s_d, s_t)
+        return [r * s_t + c for r in range(r0, r1) for c in range(c0, c1)]
+
+    def img_k(key):
+        if key < off[d]:
+            return [key]
+        a, b = divmod(key - off[d], s_d)
+        r0, r1 = orc.upscale_cell(a, s_d, s_t)
+        c0, c1 = orc.upscale_cell(b, s_d, s_t)
+        return [off[t] + r * s_t + c for r in range(r0, r1) for c in range(c0, c1)]
+
+    for qb, kb in zip(*np.nonzero(src)):
+        qs = sorted({x for q in range(qb * bq, min(qb * bq + bq, s_d * s_d)) for x in img_q(q)})
+        ks = sorted({x for k in range(kb * bk, min(kb * bk + bk, off[d + 1])) for x in img_k(k)})
+        tok[np.ix_(qs, ks)] = True
+    tok[:, :min(n_sink, l_t)] = True
+    nqb, nkb = orc.n_blocks(n_t, bq), orc.n_blocks(l_t, bk)
+    return np.array([[tok[a * bq:(a + 1) * bq, b * bk:(b + 1) * bk].any() for b in range(nkb)]
+                     for a in range(nqb)])
+
+
+@pytest.mark.parametrize("sides,d,t,bq,bk,sink", [
+    ((1, 2, 4, 6, 8), 2, 4, 4, 4, 1),
+    ((1, 2, 4, 6, 8), 3, 4, 8, 4, 5),
+    ((1, 2, 3, 5, 7), 2, 4, 4, 8, 0),
+    ((1, 2, 4, 6, 8, 12), 3, 5, 16, 16, 21),
+])
+def test_map_2d_matches_token_level(sides, d, t, bq, bk, sink):
+    off = orc.scale_offsets(sides)
+    rng = np.random.default_rng(d * 10 + t)
+    src = rng.random((orc.n_blocks(sides[d] ** 2, bq), orc.n_blocks(off[d + 1], bk))) < 0.35
+    dst = orc.map_block_mask_2d(src, sides, d, t, bq, bk, sink)
+    assert np.array_equal(dst, _token_level_2d(src, sides, d, t, bq, bk, sink))
+
+
+def test_map_2d_identity_and_invariants():
+    sides = inputs.INFINITY_SIDES
+    off = orc.scale_offsets(sides)
+    rng = np.random.default_rng(11)
+    src = rng.random((8, 20)) < 0.3
+    # same scale: every token maps to itself
+    assert np.array_equal(orc.map_block_mask_2d(src, sides, 9, 9, 128, 128, 0), src)
+    dst = orc.map_block_mask_2d(src, sides, 9, 12, 128, 128, 121)
+    assert dst[:, 0].all()
+    # keys of the scales strictly between the two are reached only by the sink
+    mid = [kb for kb in range(83) if kb * 128 >= off[10] and (kb + 1) * 128 <= off[12]]
+    assert mid and not dst[:, mid].any()
+    # a full source covers the earlier scales and the target's own scale, for every query block
+    full = orc.map_block_mask_2d(np.ones((8, 20), bool), sides, 9, 12, 128, 128, 0)
+    keep = [kb for kb in range(83) if kb * 128 < off[9] or (kb + 1) * 128 > off[12]]
+    assert full[:, keep].all()
+    # monotone in the source
+    more = src | (rng.random((8, 20)) < 0.2)
+    assert np.all(orc.map_block_mask_2d(more, sides, 9, 12, 128, 128, 121) >= dst)
+    cnt, idx, blk = orc.map_indices_2d(*orc.block_lists(src), sides, 9, 12, 128, 128, 121)
+    assert np.array_equal(blk, dst)
