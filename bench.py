@@ -346,7 +346,8 @@ def main():
             from block_sparse_cross_sparvar_b200 import workloads
             del q, kk, vv, o, hq, hk, hv
             torch.cuda.empty_cache()
-            for fn in (workloads.cs4a_full_pass, workloads.csla_radius_sweep, workloads.density_sweep):
+            for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass,
+                       workloads.csla_radius_sweep, workloads.density_sweep):
                 print(json.dumps({"extra": fn(dev)}), flush=True)
                 torch.cuda.empty_cache()
     if world > 1:

@@ -1,6 +1,7 @@
 // Integer kernels that build and check KV-block lists:
 //   csla_mask_kernel      CSLA sink + cross-scale locality mask, one CTA per query block
 //   map_indices_kernel    CS4A proportional index mapping, one CTA per (b, h, dst query block)
+//   map_2d_kernel         CS4A scale-aware 2-D index mapping, same grid
 //   validate_lists_kernel range / order check of block lists, one warp per list
 //   coarsen_lists_kernel  fine (16/32/64) block lists -> 128x128 tile lists with
 //                         per-tile bitmasks, one CTA per (b, h, query tile)
@@ -166,6 +167,92 @@ __global__ void __launch_bounds__(kMaskThreads)
     if (tk_hi > tk_lo)
       set_bit_range(bits, static_cast<int>(tk_lo / block_kv),
                     static_cast<int>((tk_hi - 1) / block_kv));
+  }
+  if (threadIdx.x == 0 && n_sink_tok > 0)
+    set_bit_range(bits, 0, min(d_nkb - 1, (n_sink_tok - 1) / block_kv));
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int64_t drow = bh * d_nqb + qb;
+    compact_bitset(bits, d_nkb, d_idx + drow * d_nkb, d_cnt + drow,
+                   d_mask ? d_mask + drow * d_nkb : nullptr);
+  }
+}
+
+// ---------------------------------------------------------------- CS4A 2-D mapping
+// Rows (columns) [lo, hi) of a side-s_dst grid covered by row (column) i of a
+// side-s_src grid: lo = floor(i*s_dst/s_src), hi = ceil((i+1)*s_dst/s_src).
+__device__ __forceinline__ void cell_range(int64_t i, int64_t s_src, int64_t s_dst, int64_t* lo,
+                                           int64_t* hi) {
+  *lo = (i * s_dst) / s_src;
+  *hi = ((i + 1) * s_dst + s_src - 1) / s_src;
+}
+
+// A decision-scale query (i, j) (side s_d) stands for its upscaled cell of the
+// target scale (side s_t); a key below off_d keeps its index; a decision-scale
+// key (a, b) stands for its cell in the target's own tokens (from off_t).
+// Source query blocks whose cells meet this CTA's destination query block are
+// flagged first; every kept entry of a flagged block then sets the destination
+// KV blocks of its mapped keys.
+__global__ void __launch_bounds__(kMaskThreads)
+    map_2d_kernel(const int32_t* src_cnt, const int32_t* src_idx, int H, int s_d, int s_t,
+                  int off_d, int l_d, int off_t, int block_q, int block_kv, int s_nqb, int s_nkb,
+                  int d_nqb, int d_nkb, int n_sink_tok, int32_t* d_cnt, int32_t* d_idx,
+                  uint8_t* d_mask, int32_t* dev_status) {
+  extern __shared__ uint32_t bits[];
+  const int nwords = (d_nkb + 31) >> 5;
+  int* flag = reinterpret_cast<int*>(bits + nwords);
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bits[w] = 0u;
+  for (int w = threadIdx.x; w < s_nqb; w += blockDim.x) flag[w] = 0;
+  __syncthreads();
+
+  // source query blocks reaching destination tokens [a, bnd)
+  const int64_t a = static_cast<int64_t>(qb) * block_q;
+  const int64_t bnd = min(a + block_q, static_cast<int64_t>(s_t) * s_t);
+  const int n_d = s_d * s_d;
+  for (int q = threadIdx.x; q < n_d; q += blockDim.x) {
+    int64_t r0, r1, c0, c1;
+    cell_range(q / s_d, s_d, s_t, &r0, &r1);
+    cell_range(q % s_d, s_d, s_t, &c0, &c1);
+    bool hit = false;
+    for (int64_t r = r0; r < r1 && !hit; ++r) hit = (r * s_t + c0 < bnd) && (a < r * s_t + c1);
+    if (hit) flag[q / block_q] = 1;
+  }
+  __syncthreads();
+
+  for (int t = threadIdx.x; t < s_nqb * s_nkb; t += blockDim.x) {
+    const int qs = t / s_nkb, e = t % s_nkb;
+    const int64_t srow = bh * s_nqb + qs;
+    int cnt = src_cnt[srow];
+    if (cnt < 0 || cnt > s_nkb) {
+      if (e == 0 && dev_status) atomicOr(dev_status, 0x1);
+      cnt = cnt < 0 ? 0 : s_nkb;
+    }
+    if (e >= cnt || !flag[qs]) continue;
+    const int kb = src_idx[srow * s_nkb + e];
+    if (kb < 0 || kb >= s_nkb) {
+      if (dev_status) atomicOr(dev_status, 0x1);
+      continue;
+    }
+    const int klo = kb * block_kv, khi = min(klo + block_kv, l_d);
+    // earlier scales: same keys
+    const int ihi = min(khi, off_d);
+    if (ihi > klo) set_bit_range(bits, klo / block_kv, (ihi - 1) / block_kv);
+    // decision-scale keys: their cells in the target scale's own tokens
+    const int u0 = max(klo, off_d) - off_d, u1 = khi - off_d;
+    for (int row = u0 / s_d; u1 > u0 && row <= (u1 - 1) / s_d; ++row) {
+      const int b0 = row == u0 / s_d ? u0 % s_d : 0;
+      const int b1 = row == (u1 - 1) / s_d ? (u1 - 1) % s_d : s_d - 1;
+      int64_t r0, r1, c0, c1, cx, cy;
+      cell_range(row, s_d, s_t, &r0, &r1);
+      cell_range(b0, s_d, s_t, &c0, &cx);
+      cell_range(b1, s_d, s_t, &cy, &c1);
+      for (int64_t r = r0; r < r1; ++r) {
+        const int64_t k0 = off_t + r * s_t + c0, k1 = off_t + r * s_t + c1 - 1;
+        set_bit_range(bits, static_cast<int>(k0 / block_kv), static_cast<int>(k1 / block_kv));
+      }
+    }
   }
   if (threadIdx.x == 0 && n_sink_tok > 0)
     set_bit_range(bits, 0, min(d_nkb - 1, (n_sink_tok - 1) / block_kv));

@@ -242,6 +242,44 @@ int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_idx, int B, i
   return SPARVAR_OK;
 }
 
+int sparvar_map_indices_2d(const int32_t* src_cnt, const int32_t* src_idx, int B, int H,
+                           const int32_t* sides, int n_scales, int src_scale, int dst_scale,
+                           int block_q, int block_kv, int n_sink_tokens, int32_t* dst_cnt,
+                           int32_t* dst_idx, uint8_t* dst_blk_mask, int32_t* dev_status,
+                           void* stream) {
+  sparvar::ScaleGeometry g;
+  int rc = build_geometry(sides, n_scales, &g);
+  if (rc) return rc;
+  if (!src_cnt || !src_idx || !dst_cnt || !dst_idx)
+    return fail(SPARVAR_ERR_INVALID_ARG, "list pointer is NULL");
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (src_scale < 0 || dst_scale < src_scale || dst_scale >= n_scales)
+    return fail(SPARVAR_ERR_INVALID_ARG, "scales %d -> %d: need 0 <= src <= dst < %d", src_scale,
+                dst_scale, n_scales);
+  if (!block_ok(block_q) || !block_ok(block_kv))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "block sizes (%d, %d) not in {16, 32, 64, 128}", block_q,
+                block_kv);
+  if (n_sink_tokens < 0) return fail(SPARVAR_ERR_INVALID_ARG, "n_sink_tokens < 0");
+  const int s_d = g.side[src_scale], s_t = g.side[dst_scale];
+  const int s_nqb = static_cast<int>(ceil_div(static_cast<int64_t>(s_d) * s_d, block_q));
+  const int s_nkb = static_cast<int>(ceil_div(g.off[src_scale + 1], block_kv));
+  const int d_nqb = static_cast<int>(ceil_div(static_cast<int64_t>(s_t) * s_t, block_q));
+  const int d_nkb = static_cast<int>(ceil_div(g.off[dst_scale + 1], block_kv));
+  const size_t smem = static_cast<size_t>((d_nkb + 31) / 32) * 4 + static_cast<size_t>(s_nqb) * 4;
+  if (smem > 48 * 1024) return fail(SPARVAR_ERR_UNSUPPORTED, "block grids too large");
+  if (static_cast<int64_t>(s_nqb) * s_nkb > (1ll << 30))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "source block grid too large");
+  dim3 grid(d_nqb, H, B);
+  sparvar::map_2d_kernel<<<grid, sparvar::kMaskThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      src_cnt, src_idx, H, s_d, s_t, g.off[src_scale], g.off[src_scale + 1], g.off[dst_scale],
+      block_q, block_kv, s_nqb, s_nkb, d_nqb, d_nkb, n_sink_tokens, dst_cnt, dst_idx,
+      dst_blk_mask, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "map_2d_kernel launch");
+  return SPARVAR_OK;
+}
+
 int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_idx,
                           const int64_t* list_strides, int idx_row_len, int B, int H, int Lq,
                           int Lkv, int block, int32_t* tile_cnt, int32_t* tile_idx,

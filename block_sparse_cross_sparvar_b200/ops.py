@@ -39,6 +39,8 @@ EXPORTS = {
     "sparvar_block_sparse_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p,
                                        _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _i, _i, _i, _f, _vp,
                                        _vp], _i),
+    "sparvar_map_indices_2d": ([_vp, _vp, _i, _i, _i32p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                _vp, _vp], _i),
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
@@ -240,6 +242,34 @@ def sparvar_map_indices(src_cnt, src_idx, src_nq, src_lkv, dst_nq, dst_lkv, bloc
         _ptr(src_cnt), _ptr(src_idx), B, H, src_nq, src_lkv, dst_nq, dst_lkv, block_q, block_kv,
         n_sink_tokens, _ptr(cnt), _ptr(idx), _ptr(mask), _ptr(dev_status), _stream(dev)),
         "sparvar_map_indices")
+    return cnt, idx, mask
+
+
+def sparvar_map_indices_2d(src_cnt, src_idx, sides, src_scale, dst_scale, block_q=128,
+                           block_kv=128, n_sink_tokens=0, with_mask=False, dev_status=None):
+    """CS4A scale-aware 2-D mapping of [B, H, NQB_src] lists from scale src_scale to
+    dst_scale of the schedule ``sides``: (cnt, idx, mask|None)."""
+    if src_cnt.dim() != 3 or not src_cnt.is_contiguous() or not src_idx.is_contiguous():
+        raise SparvarError("src_cnt must be contiguous [B, H, NQB_src]; src_idx contiguous")
+    B, H, s_nqb = src_cnt.shape
+    off = [0]
+    for s in sides:
+        off.append(off[-1] + s * s)
+    if s_nqb != -(-sides[src_scale] ** 2 // block_q):
+        raise SparvarError("src_cnt does not match the source scale's query blocks")
+    s_nkb = -(-off[src_scale + 1] // block_kv)
+    if src_idx.shape != (B, H, s_nqb, s_nkb):
+        raise SparvarError(f"src_idx must be [B, H, {s_nqb}, {s_nkb}]")
+    d_nqb, d_nkb = -(-sides[dst_scale] ** 2 // block_q), -(-off[dst_scale + 1] // block_kv)
+    dev = src_cnt.device
+    cnt = torch.empty(B, H, d_nqb, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, H, d_nqb, d_nkb, dtype=torch.int32, device=dev)
+    mask = torch.empty(B, H, d_nqb, d_nkb, dtype=torch.uint8, device=dev) if with_mask else None
+    arr = (ctypes.c_int32 * len(sides))(*sides)
+    _check(lib().sparvar_map_indices_2d(
+        _ptr(src_cnt), _ptr(src_idx), B, H, arr, len(sides), src_scale, dst_scale, block_q,
+        block_kv, n_sink_tokens, _ptr(cnt), _ptr(idx), _ptr(mask), _ptr(dev_status), _stream(dev)),
+        "sparvar_map_indices_2d")
     return cnt, idx, mask
 
 

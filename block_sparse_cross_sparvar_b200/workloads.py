@@ -3,7 +3,8 @@
 * ``cs4a_full_pass``: all 13 scales of one generation step with CS4A: scales
   1-10 dense (the 32x32 scale also yields the row LSE), the decision on the
   32x32 scale (pooled mass >= 0.95), and the mapped lists for 40x40, 48x48 and
-  64x64.
+  64x64; ``cs4a_topk_2d_pass`` the same with the Top-K rule (ratio 0.2) and the
+  scale-aware 2-D mapping.
 * ``csla_radius_sweep``: the Infinity-8B-like last two scales (B2 H32) with the
   CSLA locality radius of earlier scales at 1, 2 and 4.
 * ``density_sweep``: the last scale with random block lists at fixed densities
@@ -66,7 +67,13 @@ def time_ms(fn, reps, device, warmup=3):
     return float(np.median(out))
 
 
-def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision_scale=9):
+def cs4a_topk_2d_pass(device, reps=10, seed=0):
+    """The 13-scale pass with the Top-K rule (ratio 0.2) and the 2-D mapping."""
+    return cs4a_full_pass(device, reps, seed, topk_ratio=0.2, mapping="2d")
+
+
+def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision_scale=9,
+                   topk_ratio=0.0, mapping="1d"):
     sides = inputs.INFINITY_SIDES
     d = inputs.make_qkv(seed, B, H, sides, D, 5)
     off = d["offsets"]
@@ -87,7 +94,7 @@ def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision
             cnt, idx = dense[s]
             if s == decision_scale:
                 _, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=outs[s], return_lse=True)
-                dc, di, _ = ops.sparvar_decide_blocks(q, k, tau, lse=lse)
+                dc, di, _ = ops.sparvar_decide_blocks(q, k, tau, lse=lse, topk_ratio=topk_ratio)
                 state["dec"] = (dc, di)
             else:
                 ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=outs[s])
@@ -95,7 +102,11 @@ def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision
         src_nq, src_lkv = off[decision_scale + 1] - off[decision_scale], off[decision_scale + 1]
         for s in range(decision_scale + 1, n_scales):
             nq, L = off[s + 1] - off[s], off[s + 1]
-            mc, mi, _ = ops.sparvar_map_indices(dc, di, src_nq, src_lkv, nq, L, 128, 128, off[5])
+            if mapping == "2d":
+                mc, mi, _ = ops.sparvar_map_indices_2d(dc, di, sides, decision_scale, s, 128, 128,
+                                                       off[5])
+            else:
+                mc, mi, _ = ops.sparvar_map_indices(dc, di, src_nq, src_lkv, nq, L, 128, 128, off[5])
             state[s] = (mc, mi)
             ops.sparvar_block_sparse_attn_fwd(q_all[:, :, off[s]:off[s + 1]], k_all[:, :, :L],
                                               v_all[:, :, :L], mc, mi, out=outs[s])
@@ -112,7 +123,9 @@ def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision
         per_scale[f"{sides[s]}x{sides[s]}"] = {"gflop": f / 1e9,
                                                 "density": f / (4 * nq * L * D * B * H)}
         flops += f
-    return {"workload": "cs4a_full_pass_13_scales", "B": B, "H": H, "D": D, "tau": tau,
+    rule = f"topk {topk_ratio}" if topk_ratio > 0 else f"mass {tau}"
+    return {"workload": f"cs4a_full_pass_13_scales_{mapping}_mapping", "B": B, "H": H, "D": D,
+            "selection": rule,
             "ms": ms, "gflop": flops / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
             "scales": per_scale}
 

@@ -163,6 +163,38 @@ SPARVAR_API int sparvar_map_indices(const int32_t* src_cnt, const int32_t* src_i
                         uint8_t* dst_blk_mask, int32_t* dev_status, void* stream);
 
 /*
+ * CS4A cross-scale index mapping, scale-aware 2-D reading ("Methodology in
+ * Plain English", CS4A paragraph: kept positions rescaled to a later, larger
+ * scale, which the pages call scale self-similar; this library's alternative
+ * to the proportional 1-D reading of sparvar_map_indices).
+ *
+ * On the schedule `sides` (host, n_scales int32), the decision scale src_scale
+ * (side s_d) and a target dst_scale >= src_scale (side s_t): a decision-scale
+ * query (i, j) stands for the target queries in rows
+ * [floor(i*s_t/s_d), ceil((i+1)*s_t/s_d)) and the same range of columns; a key
+ * of a scale before src_scale keeps its index; a decision-scale key (a, b)
+ * stands for the same upscaled cell of the target scale's own tokens.  For
+ * each kept source (qb, kb) every destination (query block, KV block) holding a
+ * mapped query and a mapped key of that pair is kept; the union over kept
+ * pairs is taken and every destination KV block holding a key < n_sink_tokens
+ * is kept in every row.  Keys of the scales between the two are reached only
+ * through the sink.
+ *
+ * src_cnt  device int32 [B][H][src_nqb]; src_idx device int32 [B][H][src_nqb][src_nkb]
+ *          (src_nqb = ceil(s_d^2/block_q), src_nkb = ceil(prefix(src_scale)/block_kv)).
+ * dst_cnt  device int32 [B][H][dst_nqb]; dst_idx device int32 [B][H][dst_nqb][dst_nkb]
+ *          (dst_nqb = ceil(s_t^2/block_q), dst_nkb = ceil(prefix(dst_scale)/block_kv)),
+ *          ascending, -1 padded.  dst_blk_mask device uint8 [B][H][dst_nqb][dst_nkb] or NULL.
+ * block_q, block_kv in {16, 32, 64, 128}.  dev_status device int32 or NULL
+ * (SPARVAR_DEV_BAD_LIST for source counts or entries out of range; skipped).
+ */
+SPARVAR_API int sparvar_map_indices_2d(const int32_t* src_cnt, const int32_t* src_idx, int B,
+                                       int H, const int32_t* sides, int n_scales, int src_scale,
+                                       int dst_scale, int block_q, int block_kv, int n_sink_tokens,
+                                       int32_t* dst_cnt, int32_t* dst_idx, uint8_t* dst_blk_mask,
+                                       int32_t* dev_status, void* stream);
+
+/*
  * Block-sparse attention forward ("Key Contributions" item 3, "Main
  * Findings" block-size rows; scale-causal prefix from "What This Paper Is
  * About"):

@@ -447,3 +447,67 @@ def test_map_indices_small_blocks_and_bad_entries():
     want = [[0, 2, 3, 4], [0, 2, 3, 4], [0, 5, 6, 7], [0, 5, 6, 7]]
     for qb, w in enumerate(want):
         assert di[0, 0, qb, :dc[0, 0, qb]].tolist() == w
+
+
+# ------------------------------------------------------------------ CS4A 2-D mapping
+def _lists_from_blk(blk):
+    B, H, nqb, nkb = blk.shape
+    cnt = blk.sum(-1).astype(np.int32)
+    idx = np.full((B, H, nqb, nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                kept = np.nonzero(blk[b, h, qb])[0]
+                idx[b, h, qb, :kept.size] = kept
+    return cnt, idx
+
+
+@pytest.mark.parametrize("sides,src,dst,bq,bk,sink", [
+    (INF, 9, 10, 128, 128, 121),
+    (INF, 9, 11, 128, 128, 121),
+    (INF, 9, 12, 128, 128, 121),
+    (INF, 9, 12, 64, 64, 121),
+    (INF, 9, 9, 128, 128, 0),
+    (TINY, 3, 4, 16, 16, 5),
+    ((1, 2, 3, 5, 7, 11), 3, 5, 16, 32, 1),
+])
+def test_map_indices_2d_bit_exact(sides, src, dst, bq, bk, sink):
+    off = inputs.token_offsets(sides)
+    rng = np.random.default_rng(src * 100 + dst + bq)
+    B, H = 2, 2
+    s_nqb, s_nkb = -(-sides[src] ** 2 // bq), -(-off[src + 1] // bk)
+    blk = rng.random((B, H, s_nqb, s_nkb)) < 0.25
+    cnt, idx = _lists_from_blk(blk)
+    st = _status()
+    dc, di, dm = ops.sparvar_map_indices_2d(torch.from_numpy(cnt).cuda(),
+                                            torch.from_numpy(idx).cuda(), sides, src, dst, bq, bk,
+                                            sink, with_mask=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for b in range(B):
+        for h in range(H):
+            oc, oi, ob = orc.map_indices_2d(cnt[b, h], idx[b, h], sides, src, dst, bq, bk, sink)
+            assert np.array_equal(dc[b, h].cpu().numpy(), oc)
+            assert np.array_equal(di[b, h].cpu().numpy(), oi)
+            assert np.array_equal(dm[b, h].cpu().numpy().astype(bool), ob)
+
+
+def test_cs4a_topk_2d_pipeline_attention():
+    """Decision at the 32x32 scale with the Top-K rule, 2-D mapping to 64x64, then the
+    block-sparse attention on the mapped lists, against the oracle end to end."""
+    d = inputs.make_qkv(9, 1, 2, INF, 128, 5)
+    off = d["offsets"]
+    s, t = 9, 12
+    qd, kd = d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]]
+    dc, di, _ = ops.sparvar_decide_blocks(_dev(qd), _dev(kd), 0.95, topk_ratio=0.2)
+    mc, mi, _ = ops.sparvar_map_indices_2d(dc, di, INF, s, t, 128, 128, off[5])
+    q_bits = d["q"][:, :, off[t]:off[t + 1]]
+    kv = slice(0, off[t + 1])
+    _check_attention(q_bits, d["k"][:, :, kv], d["v"][:, :, kv], (mc, mi), 128, 128, 128,
+                     lse_check=False)
+    # the mapped lists equal the oracle's mapping of the kernel's own decision
+    dcn, din = dc.cpu().numpy(), di.cpu().numpy()
+    for h in range(2):
+        oc, oi, _ = orc.map_indices_2d(dcn[0, h], din[0, h], INF, s, t, 128, 128, off[5])
+        assert np.array_equal(mc[0, h].cpu().numpy(), oc)
+        assert np.array_equal(mi[0, h].cpu().numpy(), oi)

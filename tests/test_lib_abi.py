@@ -126,3 +126,18 @@ def test_coarsen_rejects_bad_arguments(lib):
     assert call(ls=i64(-1, 0)) == 1
     assert call(row=-1) == 1
     assert call(Lkv=4097 * 128) == 2 and "KV tiles" in lib.sparvar_last_error().decode()
+
+
+def test_map_2d_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    sides = (ctypes.c_int32 * 4)(1, 2, 4, 8)
+
+    def call(src=2, dst=3, bq=16, bk=16, sink=0, cnt=16):
+        return lib.sparvar_map_indices_2d(vp(cnt), vp(16), 1, 1, sides, 4, src, dst, bq, bk, sink,
+                                          vp(16), vp(16), vp(0), vp(0), vp(0))
+
+    assert call(src=3, dst=2) == 1 and "scales" in lib.sparvar_last_error().decode()
+    assert call(dst=4) == 1
+    assert call(bq=8) == 2
+    assert call(sink=-1) == 1
+    assert call(cnt=0) == 1
