@@ -107,13 +107,21 @@ struct Layout {
 };
 
 // One tile of this CTA's sequence, with the sequence counters at its start.
+// A tile whose predecessor (the previous non-empty tile) has at least three
+// blocks is fed by it: the predecessor's last three MMA groups issue the tile's
+// first score MMAs, and its K blocks and Q are loaded in the predecessor's ring
+// stream.  Any other non-empty tile starts with a prologue group (its first
+// score MMAs, issued once the predecessor's MMAs are done).
 struct TileCursor {
   int t;  // tile id (b * H + h) * nqb + qb; >= total when the CTA is done
   int n;  // list length (clamped to [0, idx_row_len])
   const int32_t* list;
-  int J0;    // sequence index of the tile's first block
-  int pos0;  // ring position of the tile's first operand
-  int k;     // number of non-empty tiles before this one
+  int J0;      // sequence index of the tile's first block
+  int pos0;    // ring position of the tile's first operand
+  int k;       // number of non-empty tiles before this one
+  int G;       // first MMA group of the tile
+  int prev_n;  // list length of the previous non-empty tile, -1 before the first
+  int next_n;  // list length of the next non-empty tile, 0 after the last
 };
 
 struct TileCoord {
@@ -124,34 +132,63 @@ __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
   return TileCoord{bh / a.H, bh % a.H, t % a.nqb};
 }
 
-__device__ __forceinline__ void cursor_load(TileCursor& c, const Args& a, int total, bool report) {
-  if (c.t >= total) return;
-  const TileCoord tc = tile_coord(c.t, a);
+__device__ __forceinline__ int tile_count(int t, const Args& a, bool report,
+                                          const int32_t** list) {
+  const TileCoord tc = tile_coord(t, a);
   const int64_t lrow = tc.b * a.list_sb + tc.h * a.list_sh + tc.qb;
   int n = __ldg(a.kv_cnt + lrow);
   if (n < 0 || n > a.idx_row_len) {
     if (report && a.dev_status) atomicOr(a.dev_status, 0x1);
     n = n < 0 ? 0 : a.idx_row_len;
   }
-  c.n = n;
-  c.list = a.kv_idx + lrow * a.idx_row_len;
+  if (list) *list = a.kv_idx + lrow * a.idx_row_len;
+  return n;
+}
+
+__device__ __forceinline__ void cursor_load(TileCursor& c, const Args& a, int total, bool report) {
+  if (c.t >= total) return;
+  c.n = tile_count(c.t, a, report, &c.list);
+  c.next_n = 0;
+  for (int t = c.t + gridDim.x; t < total && c.next_n == 0; t += gridDim.x)
+    c.next_n = tile_count(t, a, false, nullptr);
+}
+
+__device__ __forceinline__ bool has_prologue(const TileCursor& c) { return c.prev_n < 3; }
+__device__ __forceinline__ bool feeds_next(const TileCursor& c) { return c.n >= 3 && c.next_n > 0; }
+__device__ __forceinline__ int own_k(const TileCursor& c) { return c.n > 3 ? c.n - 3 : 0; }
+__device__ __forceinline__ int n_prologue(const TileCursor& c) {
+  return has_prologue(c) ? (c.n < 3 ? c.n : 3) : 0;
+}
+// ring positions of a tile: prologue K's, then V_j followed, when it exists, by
+// the K block whose score MMA group j issues (K_{j+3} of this tile or, for the
+// last three blocks of a feeding tile, the next tile's first K's)
+__device__ __forceinline__ bool has_k_after(const TileCursor& c, int j) {
+  return j < own_k(c) || (feeds_next(c) && j - own_k(c) < c.next_n);
+}
+__device__ __forceinline__ int ring_pos_v(const TileCursor& c, int j) {
+  const int nk = own_k(c);
+  int p = c.pos0 + n_prologue(c) + j + (j < nk ? j : nk);
+  if (feeds_next(c) && j > nk) p += (j - nk < c.next_n ? j - nk : c.next_n);
+  return p;
+}
+__device__ __forceinline__ int ring_items(const TileCursor& c) {
+  return n_prologue(c) + c.n + own_k(c) + (feeds_next(c) ? (c.next_n < 3 ? c.next_n : 3) : 0);
+}
+__device__ __forceinline__ int group_of_prologue(const TileCursor& c) { return c.G; }
+__device__ __forceinline__ int group_of_block(const TileCursor& c, int j) {
+  return c.G + (has_prologue(c) ? 1 : 0) + j;
 }
 
 __device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int total, bool report) {
   if (c.n > 0) {
-    const int n0 = c.n < 3 ? c.n : 3;
-    const int nk = c.n > 3 ? c.n - 3 : 0;
+    c.pos0 += ring_items(c);
+    c.G += c.n + (has_prologue(c) ? 1 : 0);
     c.J0 += c.n;
-    c.pos0 += n0 + c.n + nk;
     c.k += 1;
+    c.prev_n = c.n;
   }
   c.t += gridDim.x;
   cursor_load(c, a, total, report);
-}
-
-__device__ __forceinline__ int group_of_prologue(const TileCursor& c) { return c.J0 + c.k; }
-__device__ __forceinline__ int group_of_block(const TileCursor& c, int j) {
-  return c.J0 + c.k + 1 + j;
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -233,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   TileCursor first{};
   first.t = blockIdx.x;
+  first.prev_n = -1;
   cursor_load(first, args, total, threadIdx.x == 0);
 
   if (warp == kLoadWarp) {
@@ -257,29 +295,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                       tc.b);
         ++w;
       };
-      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
-        if (c.n == 0) continue;
-        const int qs = c.k & 1;
-        // Q buffer qs is free once tile k - 2's epilogue is done with it
-        if (c.k >= 2 &&
-            !mbar_wait(&bars.epi[qs], ((c.k - 2) >> 1) & 1, abort_flag, dev_status, 0x2, kWaitNs)) {
+      // Q of non-empty tile k into buffer k & 1, free once tile k - 2's epilogue is done
+      auto load_q = [&](int k, const TileCoord& tq) {
+        const int qs = k & 1;
+        if (k >= 2 &&
+            !mbar_wait(&bars.epi[qs], ((k - 2) >> 1) & 1, abort_flag, dev_status, 0x2, kWaitNs)) {
           ok = false;
-          break;
+          return;
         }
-        const TileCoord tc = tile_coord(c.t, args);
         mbar_arrive_expect_tx(&bars.q_full[qs], L::kTileBytes);
 #pragma unroll
         for (int cc = 0; cc < L::kChunks; ++cc)
-          tma_load_4d(sQ(c.k) + cc * L::kChunkBytes, &tm_q, &bars.q_full[qs], cc * 64,
-                      tc.qb * kTile, tc.h, tc.b);
+          tma_load_4d(sQ(k) + cc * L::kChunkBytes, &tm_q, &bars.q_full[qs], cc * 64,
+                      tq.qb * kTile, tq.h, tq.b);
         if (qs) ++q_issued1; else ++q_issued0;
-        const int n0 = c.n < 3 ? c.n : 3;
-        for (int jj = 0; jj < n0 && ok; ++jj)
-          produce(&tm_k, __ldg(c.list + jj), group_of_prologue(c), tc);
+      };
+      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
+        if (c.n == 0) continue;
+        const TileCoord tc = tile_coord(c.t, args);
+        if (has_prologue(c)) {
+          load_q(c.k, tc);
+          for (int jj = 0; jj < n_prologue(c) && ok; ++jj)
+            produce(&tm_k, __ldg(c.list + jj), group_of_prologue(c), tc);
+        }
+        // the next non-empty tile, when this one feeds it
+        TileCursor nx = c;
+        TileCoord tn{};
+        if (feeds_next(c)) {
+          do {
+            cursor_next(nx, args, total, false);
+          } while (nx.t < total && nx.n == 0);
+          tn = tile_coord(nx.t, args);
+        }
+        const int nk = own_k(c);
         for (int j = 0; j < c.n && ok; ++j) {
           const int grp = group_of_block(c, j);
           produce(&tm_v, __ldg(c.list + j), grp, tc);
-          if (ok && j + 3 < c.n) produce(&tm_k, __ldg(c.list + j + 3), grp, tc);
+          if (!ok) break;
+          if (j < nk) {
+            produce(&tm_k, __ldg(c.list + j + 3), grp, tc);
+          } else if (has_k_after(c, j)) {
+            if (j == nk) load_q(c.k + 1, tn);
+            if (ok) produce(&tm_k, __ldg(nx.list + (j - nk)), grp, tn);
+          }
         }
       }
       // drain: every issued TMA write lands before the CTA exits
@@ -318,15 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last1 = -1, last2 = -1;  // last two groups of the previous non-empty tile
       for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
         if (c.n == 0) continue;
-        const int n0 = c.n < 3 ? c.n : 3;
-        const int nk = c.n > 3 ? c.n - 3 : 0;
-        if (me == 0) {
+        const int nk = own_k(c);
+        if (me == 0 && has_prologue(c)) {
           // prologue: the score buffers are free once the previous tile's MMAs are done
           ok = mbar_wait(&bars.q_full[c.k & 1], (c.k >> 1) & 1, abort_flag, dev_status, 0x2,
                          kWaitNs);
           if (ok && last1 >= 0) ok = wait_group(bars.rel, last1, abort_flag, dev_status);
           if (ok && last2 >= 0) ok = wait_group(bars.rel, last2, abort_flag, dev_status);
-          for (int jj = 0; jj < n0 && ok; ++jj) {
+          for (int jj = 0; jj < n_prologue(c) && ok; ++jj) {
             wait_pos(c.pos0 + jj);
             if (!ok) break;
             tc_fence_after();
@@ -339,10 +396,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = ((c.J0 & 1) == me) ? 0 : 1; j < c.n && ok; j += 2) {
           const int J = c.J0 + j;
           ok = mbar_wait(&bars.p_full[J % 3], (J / 3) & 1, abort_flag, dev_status, 0x2, kWaitNs);
-          const int pv = c.pos0 + n0 + j + (j < nk ? j : nk);
-          const bool more = j + 3 < c.n;
+          const int pv = ring_pos_v(c, j);
+          const bool more = has_k_after(c, j);
+          const bool feed = more && j >= nk;  // S of the next tile's block j - nk
           wait_pos(pv);
           if (more) wait_pos(pv + 1);
+          if (feed)
+            ok = ok && mbar_wait(&bars.q_full[(c.k + 1) & 1], ((c.k + 1) >> 1) & 1, abort_flag,
+                                 dev_status, 0x2, kWaitNs);
           if (!ok) break;
           const uint64_t dvs = dv + static_cast<uint64_t>((pv % NS) * kBufStep);
           const uint32_t a_col = tmem + (J % 3) * 128;
@@ -353,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    idesc_pv, 1u);
           if (more) {
             // buffer J mod 3 is free once PV_J has read P_J (this issuer's MMAs run in order)
-            issue_s(J + 3, c.k, pv + 1);
+            issue_s(J + 3, feed ? c.k + 1 : c.k, pv + 1);
             mma_commit(&bars.s_full[J % 3]);
           }
           mma_commit(&bars.rel[group_of_block(c, j) % kRel]);

@@ -4,23 +4,26 @@ A small discrete model of the persistent attn_fwd_kernel.cuh: one CTA walking
 several query tiles with the TMA producer, the two MMA issuers, the two softmax
 groups and the tensor core, connected by mbarriers with phase counters.
 Random interleavings (and random "raise the reference max" decisions) are
-explored for many tile sequences (empty tiles included) and ring sizes,
-checking
+explored for many tile sequences (empty and short tiles included) and ring
+sizes, checking
 
 * that no schedule deadlocks, and
 * that every parity wait only ever observes its own phase or the next one
   (a barrier two phases ahead would make `try_wait.parity` lie).
 
 The model follows the kernel's protocol step for step: block J of the CTA's
-sequence goes to softmax group and issuer J mod 2, a tile's prologue group
-(its first score MMAs) is issued by issuer 0 after the previous tile's MMAs,
-MMA group G commits on rel[G mod 16], an issuer waits for its block's P
-before the block's V and K ring slots (a slot may be two loads behind before
-then), the producer waits for the group that last used a ring slot, and Q
-buffers alternate between non-empty tiles with an epilogue hand-back.  Known-bad variants (waiting for P of the next block
-inside the current MMA group; fewer release barriers than the protocol needs;
-waiting for the ring slots before P) are checked to fail, so the checker is
-not vacuous.
+sequence goes to softmax group and issuer J mod 2; MMA group J is PV_J then
+the score MMA of block J + 3, also across a tile boundary when the tile has at
+least three blocks (it then feeds the next tile: the next tile's Q and first
+K blocks are loaded in its ring stream); a tile whose predecessor is shorter
+starts with a prologue group issued by issuer 0 after the predecessor's MMAs;
+groups commit on rel[G mod 16]; an issuer waits for its block's P before the
+block's V and K ring slots (a slot may be two loads behind before then); the
+producer waits for the group that last used a ring slot; Q buffers alternate
+between non-empty tiles and come back after each tile's epilogue.  Known-bad
+variants (waiting for P of the next block inside the current MMA group; fewer
+release barriers than the protocol needs; waiting for ring slots before P) are
+checked to fail, so the checker is not vacuous.
 """
 import random
 
@@ -38,10 +41,32 @@ class Bar:
             self.done += 1
 
 
+def plan(tiles):
+    """Per non-empty tile: first block J0, tile number k, prologue flag, groups."""
+    desc, J0, k, G, prev_n = [], 0, 0, 0, None
+    for n in tiles:
+        if n == 0:
+            continue
+        d = dict(n=n, J0=J0, k=k, pro=prev_n is None or prev_n < 3, n0=min(n, 3))
+        if d["pro"]:
+            d["Gpro"] = G
+            G += 1
+        d["G0"] = G  # group of block j is G0 + j
+        G += n
+        desc.append(d)
+        J0, k, prev_n = J0 + n, k + 1, n
+    for i, d in enumerate(desc):
+        d["next"] = desc[i + 1] if i + 1 < len(desc) else None
+        d["feeds"] = d["next"] is not None and not d["next"]["pro"]
+    return desc
+
+
 class Model:
-    def __init__(self, tiles, ns, p_raise, seed, n_rel=16, bad_next_p=False, bad_slots_first=False):
+    def __init__(self, tiles, ns, p_raise, seed, n_rel=16, bad_next_p=False,
+                 bad_slots_first=False):
         self.rng = random.Random(seed)
         self.ns, self.p_raise, self.n_rel = ns, p_raise, n_rel
+        self.bad_slots_first = bad_slots_first
         self.bars = {"drain": Bar(2)}
         for i in range(2):
             self.bars[f"q_full{i}"] = Bar()
@@ -53,31 +78,43 @@ class Model:
         for i in range(3):
             self.bars[f"s_full{i}"] = Bar()
             self.bars[f"p_full{i}"] = Bar()
-        # per-tile sequence counters, as the kernel's cursor advances them
-        self.desc = []
-        J0 = pos0 = k = 0
-        for n in tiles:
-            n0, nk = min(n, 3), max(n - 3, 0)
-            self.desc.append(dict(n=n, J0=J0, pos0=pos0, k=k, n0=n0, nk=nk))
-            if n > 0:
-                J0, pos0, k = J0 + n, pos0 + n0 + n + nk, k + 1
+        self.desc = plan(tiles)
+        self.items = self.ring_items()
+        self.pos = {}
+        p = 0
+        for kind, x, _ in self.items:
+            if kind != "Q":
+                self.pos[(kind, x)] = p
+                p += 1
         self.tc, self.tma, self.passed = [], [], set()
-        self.bad_slots_first = bad_slots_first
         issuer = self.issuer_bad if bad_next_p else self.issuer
         self.roles = [self.loader(), issuer(0), issuer(1), self.softmax(0), self.softmax(1)]
         self.cur = [next(r) for r in self.roles]
 
     @staticmethod
-    def pos_v(d, j):
-        return d["pos0"] + d["n0"] + j + min(j, d["nk"])
+    def k_after(d, j):
+        """Block whose K follows V_j in the ring, or None."""
+        if j + 3 < d["n"]:
+            return d["J0"] + j + 3
+        if d["feeds"] and j + 3 - d["n"] < d["next"]["n"]:
+            return d["J0"] + j + 3
+        return None
 
-    @staticmethod
-    def group(d, j):  # MMA group of block j of tile d
-        return d["J0"] + d["k"] + 1 + j
-
-    @staticmethod
-    def prologue_group(d):
-        return d["J0"] + d["k"]
+    def ring_items(self):
+        items = []
+        for d in self.desc:
+            if d["pro"]:
+                items.append(("Q", d["k"], None))
+                items += [("K", d["J0"] + jj, d["Gpro"]) for jj in range(d["n0"])]
+            for j in range(d["n"]):
+                g = d["G0"] + j
+                items.append(("V", d["J0"] + j, g))
+                x = self.k_after(d, j)
+                if x is not None:
+                    if j + 3 == d["n"]:
+                        items.append(("Q", d["next"]["k"], None))
+                    items.append(("K", x, g))
+        return items
 
     def rel(self, g):
         return ("wait", f"rel{g % self.n_rel}", g // self.n_rel)
@@ -86,66 +123,57 @@ class Model:
         return ("wait", f"full{p % self.ns}", p // self.ns)
 
     def loader(self):
-        owner = [None] * self.ns  # group that frees each slot
-        w = 0
-        for d in self.desc:
-            if d["n"] == 0:
+        owner, w = [None] * self.ns, 0
+        for kind, x, g in self.items:
+            if kind == "Q":
+                if x >= 2:
+                    yield ("wait", f"epi{x % 2}", (x - 2) // 2)
+                yield ("tma", f"q_full{x % 2}")
                 continue
-            k = d["k"]
-            if k >= 2:
-                yield ("wait", f"epi{k % 2}", (k - 2) // 2)
-            yield ("tma", f"q_full{k % 2}")
-            items = [self.prologue_group(d)] * d["n0"]
-            for j in range(d["n"]):
-                items.append(self.group(d, j))  # V_j
-                if j + 3 < d["n"]:
-                    items.append(self.group(d, j))  # K_{j+3}
-            for g in items:
-                s = w % self.ns
-                if owner[s] is not None:
-                    yield self.rel(owner[s])
-                owner[s] = g
-                yield ("tma", f"full{s}")
-                w += 1
+            s = w % self.ns
+            if owner[s] is not None:
+                yield self.rel(owner[s])
+            owner[s] = g
+            yield ("tma", f"full{s}")
+            w += 1
         yield ("end",)
 
     def prologue(self, d, prev):
         yield ("wait", f"q_full{d['k'] % 2}", d["k"] // 2)
         if prev is not None:
-            yield self.rel(self.group(prev, prev["n"] - 1))
+            yield self.rel(prev["G0"] + prev["n"] - 1)
             if prev["n"] >= 2:
-                yield self.rel(self.group(prev, prev["n"] - 2))
+                yield self.rel(prev["G0"] + prev["n"] - 2)
         for jj in range(d["n0"]):
-            yield self.full(d["pos0"] + jj)
+            yield self.full(self.pos[("K", d["J0"] + jj)])
             yield ("issue",)
             yield ("commit", f"s_full{(d['J0'] + jj) % 3}")
-        yield ("commit", f"rel{self.prologue_group(d) % self.n_rel}")
+        yield ("commit", f"rel{d['Gpro'] % self.n_rel}")
 
     def issuer(self, me):
         prev = None
         for d in self.desc:
-            n = d["n"]
-            if n == 0:
-                continue
-            if me == 0:
+            if d["pro"] and me == 0:
                 yield from self.prologue(d, prev)
-            for j in range(n):
-                J = d["J0"] + j
-                if J % 2 != me:
+            for j in range(d["n"]):
+                X = d["J0"] + j
+                if X % 2 != me:
                     continue
-                pv = self.pos_v(d, j)
+                x = self.k_after(d, j)
                 if not self.bad_slots_first:
-                    yield ("wait", f"p_full{J % 3}", J // 3)
-                yield self.full(pv)
-                if j + 3 < n:
-                    yield self.full(pv + 1)
+                    yield ("wait", f"p_full{X % 3}", X // 3)
+                yield self.full(self.pos[("V", X)])
+                if x is not None:
+                    yield self.full(self.pos[("K", x)])
+                    if j + 3 >= d["n"]:
+                        yield ("wait", f"q_full{d['next']['k'] % 2}", d["next"]["k"] // 2)
                 if self.bad_slots_first:
-                    yield ("wait", f"p_full{J % 3}", J // 3)
+                    yield ("wait", f"p_full{X % 3}", X // 3)
                 yield ("issue",)
-                if j + 3 < n:
+                if x is not None:
                     yield ("issue",)
-                    yield ("commit", f"s_full{J % 3}")
-                yield ("commit", f"rel{self.group(d, j) % self.n_rel}")
+                    yield ("commit", f"s_full{X % 3}")
+                yield ("commit", f"rel{(d['G0'] + j) % self.n_rel}")
             prev = d
         yield ("commit", "drain")
         yield ("wait", "drain", 0)
@@ -160,23 +188,23 @@ class Model:
             return
         prev = None
         for d in self.desc:
-            n = d["n"]
-            if n == 0:
-                continue
-            yield from self.prologue(d, prev)
+            if d["pro"]:
+                yield from self.prologue(d, prev)
             yield ("wait", f"p_full{d['J0'] % 3}", d["J0"] // 3)
-            for j in range(n):
-                J = d["J0"] + j
+            for j in range(d["n"]):
+                X = d["J0"] + j
                 yield ("issue",)
-                if j + 1 < n:
-                    yield ("wait", f"p_full{(J + 1) % 3}", (J + 1) // 3)
-                pv = self.pos_v(d, j)
-                yield self.full(pv)
-                if j + 3 < n:
-                    yield self.full(pv + 1)
+                if j + 1 < d["n"]:
+                    yield ("wait", f"p_full{(X + 1) % 3}", (X + 1) // 3)
+                yield self.full(self.pos[("V", X)])
+                x = self.k_after(d, j)
+                if x is not None:
+                    yield self.full(self.pos[("K", x)])
+                    if j + 3 >= d["n"]:
+                        yield ("wait", f"q_full{d['next']['k'] % 2}", d["next"]["k"] // 2)
                     yield ("issue",)
-                    yield ("commit", f"s_full{J % 3}")
-                yield ("commit", f"rel{self.group(d, j) % self.n_rel}")
+                    yield ("commit", f"s_full{X % 3}")
+                yield ("commit", f"rel{(d['G0'] + j) % self.n_rel}")
             prev = d
         yield ("commit", "drain")
         yield ("wait", "drain", 0)
@@ -184,26 +212,26 @@ class Model:
 
     def softmax(self, g):
         for u, d in enumerate(self.desc):
-            n = d["n"]
-            for j in range(n):
-                J = d["J0"] + j
-                if J % 2 != g:
+            for j in range(d["n"]):
+                X = d["J0"] + j
+                if X % 2 != g:
                     continue
-                yield ("wait", f"s_full{J % 3}", J // 3)
-                if J > 0:
-                    yield ("wait", f"p_full{(J - 1) % 3}", (J - 1) // 3)
+                yield ("wait", f"s_full{X % 3}", X // 3)
+                if X > 0:
+                    yield ("wait", f"p_full{(X - 1) % 3}", (X - 1) // 3)
                 if j > 0 and self.rng.random() < self.p_raise:
                     # O rescale: the latest group of each issuer must have completed
-                    yield self.rel(self.group(d, j - 1))
+                    yield self.rel(d["G0"] + j - 1)
                     if j > 1:
-                        yield self.rel(self.group(d, j - 2))
-                yield ("arrive", f"p_full{J % 3}")
-            if n > 0:  # epilogue: every MMA of the tile has completed
-                yield self.rel(self.group(d, n - 1))
-                if n >= 2:
-                    yield self.rel(self.group(d, n - 2))
-            yield ("bar", u)  # 256-thread named barrier of both groups
-            if g == 0 and n > 0:
+                        yield self.rel(d["G0"] + j - 2)
+                yield ("arrive", f"p_full{X % 3}")
+            # epilogue: every MMA of the tile has completed, then a named barrier of
+            # both groups, then the Q buffer goes back to the producer
+            yield self.rel(d["G0"] + d["n"] - 1)
+            if d["n"] >= 2:
+                yield self.rel(d["G0"] + d["n"] - 2)
+            yield ("bar", u)
+            if g == 0:
                 yield ("arrive", f"epi{d['k'] % 2}")
         yield ("end",)
 
@@ -218,7 +246,7 @@ class Model:
         assert op[2] <= done <= op[2] + 1, f"parity ambiguity on {op[1]}: phase {op[2]}, done {done}"
         return done == op[2] + 1
 
-    def run(self, max_steps=400000):
+    def run(self, max_steps=500000):
         for _ in range(max_steps):
             live = [i for i, op in enumerate(self.cur) if op[0] != "end"]
             if not live and not self.tc and not self.tma:
@@ -254,18 +282,25 @@ class Model:
 def _tile_sequences(seed, count):
     rng = random.Random(seed)
     seqs = [[n] for n in list(range(0, 26)) + [41, 83]]
-    seqs += [[0, 0], [1, 1, 1, 1, 1], [2, 0, 2, 0, 2], [3, 21, 3, 21]]
+    seqs += [[0, 0], [1, 1, 1, 1, 1], [2, 0, 2, 0, 2], [3, 21, 3, 21], [3, 3, 3, 3],
+             [21, 1, 21, 2, 21, 3, 21], [4, 0, 0, 5, 2, 3]]
     for _ in range(count):
-        seqs.append([rng.choice([0, 1, 2, 3, 4, 5, 7, 9, 15, 21]) for _ in range(rng.randint(2, 7))])
+        seqs.append([rng.choice([0, 1, 2, 3, 4, 5, 7, 9, 15, 21]) for _ in range(rng.randint(2, 8))])
     return seqs
 
 
 @pytest.mark.parametrize("ns", [5, 12])
 @pytest.mark.parametrize("p_raise", [0.0, 0.3, 1.0])
 def test_protocol_never_deadlocks(ns, p_raise):
-    for t, tiles in enumerate(_tile_sequences(ns * 10 + int(p_raise * 10), 60)):
+    for t, tiles in enumerate(_tile_sequences(ns * 10 + int(p_raise * 10), 80)):
         for seed in range(4):
             assert Model(tiles, ns, p_raise, seed * 1000 + t).run(), (tiles, seed)
+
+
+def test_fed_and_prologue_tiles():
+    desc = plan([21, 2, 5, 0, 3, 1])
+    assert [d["pro"] for d in desc] == [True, False, True, False, False]
+    assert [d["feeds"] for d in desc] == [True, False, True, True, False]
 
 
 def test_known_bad_next_p_wait_is_caught():
