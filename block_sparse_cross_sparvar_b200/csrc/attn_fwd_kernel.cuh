@@ -36,10 +36,12 @@
 // m (block max more than 2^8 above it: O is rescaled in place once the tile's
 // earlier PVs have completed) or, if m moved meanwhile, rescales its own P in
 // TMEM.  O is zeroed before a tile's first PV, so the two issuers' PVs may
-// accumulate in either order.  Each block's softmax takes two passes over S in
+// accumulate in either order.  Each issuer signs o_done after its last PV of a
+// tile, so the epilogue need not wait for the next tile's score MMAs issued in
+// the same groups.  Each block's softmax takes two passes over S in
 // TMEM: the row max, then P in packed f32x2 arithmetic from the 96 columns kept
-// in registers plus the last 32 re-read.  The epilogue waits for the tile's
-// last two groups, merges the two groups' row sums against the final m
+// in registers plus the last 32 re-read.  The epilogue waits for o_done,
+// merges the two groups' row sums against the final m
 // (exchanging them through the tile's Q buffer, which no MMA reads any more),
 // stages the normalised bf16 output in that buffer in the output tensor map's
 // swizzled layout, sends it with one TMA store per 64 columns, writes the LSE,
@@ -92,6 +94,7 @@ struct __align__(8) Bars {
   uint64_t full[kMaxSlots];       // ring slot loaded (TMA transaction count)
   uint64_t rel[kRel];             // MMA group G done: [G % kRel], phase G / kRel
   uint64_t s_full[3], p_full[3];  // block J: [J % 3], phase J / 3
+  uint64_t o_done[2];             // every PV of non-empty tile k done: [k & 1], phase k >> 1
   uint64_t drain;
 };
 
@@ -246,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 128);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&bars.o_done[i], 2);  // one commit per issuer
     mbar_init(&bars.drain, 2);  // one commit per issuer
     fence_barrier_init();
   }
@@ -412,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kTile / 16; ++kk)
             mma_ts(tmem + kColO, a_col + kk * 8, dvs + static_cast<uint64_t>(kk * (2048 >> 4)),
                    idesc_pv, 1u);
+          // this issuer's last PV of the tile: O is final once both issuers' are done
+          if (j + 2 >= c.n) mma_commit(&bars.o_done[c.k & 1]);
           if (more) {
             // buffer J mod 3 is free once PV_J has read P_J (this issuer's MMAs run in order)
             issue_s(J + 3, feed ? c.k + 1 : c.k, pv + 1);
@@ -419,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&bars.rel[group_of_block(c, j) % kRel]);
         }
+        // an issuer with no block in this (one-block) tile still signs for O
+        if (ok && c.n == 1 && ((c.J0 & 1) != me)) mma_commit(&bars.o_done[c.k & 1]);
         last1 = group_of_block(c, c.n - 1);
         last2 = c.n >= 2 ? group_of_block(c, c.n - 2) : -1;
       }
@@ -629,11 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ---- epilogue of the tile
-      if (good && c.n > 0) {
-        good = warp_wait_group(bars.rel, group_of_block(c, c.n - 1), abort_flag, dev_status) &&
-               (c.n < 2 ||
-                warp_wait_group(bars.rel, group_of_block(c, c.n - 2), abort_flag, dev_status));
-      }
+      if (good && c.n > 0)
+        good = warp_wait(&bars.o_done[c.k & 1], (c.k >> 1) & 1, abort_flag, dev_status);
       // every MMA of the tile is done and its Q buffer is free: it takes first the two
       // groups' sums, then the bf16 output tile, which leaves through a TMA store
       uint8_t* qbuf = smem_gen + L::kQ + (c.k & 1) * L::kTileBytes;

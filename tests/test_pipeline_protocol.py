@@ -17,10 +17,12 @@ the score MMA of block J + 3, also across a tile boundary when the tile has at
 least three blocks (it then feeds the next tile: the next tile's Q and first
 K blocks are loaded in its ring stream); a tile whose predecessor is shorter
 starts with a prologue group issued by issuer 0 after the predecessor's MMAs;
-groups commit on rel[G mod 16]; an issuer waits for its block's P before the
-block's V and K ring slots (a slot may be two loads behind before then); the
-producer waits for the group that last used a ring slot; Q buffers alternate
-between non-empty tiles and come back after each tile's epilogue.  Known-bad
+groups commit on rel[G mod 16] and each issuer signs a per-tile o_done after
+its last PV of the tile, which the epilogue waits for; an issuer waits for its
+block's P before the block's V and K ring slots (a slot may be two loads
+behind before then); the producer waits for the group that last used a ring
+slot; Q buffers alternate between non-empty tiles and come back after each
+tile's epilogue.  Known-bad
 variants (waiting for P of the next block inside the current MMA group; fewer
 release barriers than the protocol needs; waiting for ring slots before P) are
 checked to fail, so the checker is not vacuous.
@@ -71,6 +73,7 @@ class Model:
         for i in range(2):
             self.bars[f"q_full{i}"] = Bar()
             self.bars[f"epi{i}"] = Bar()
+            self.bars[f"o_done{i}"] = Bar(2)
         for i in range(ns):
             self.bars[f"full{i}"] = Bar()
         for i in range(n_rel):
@@ -170,10 +173,14 @@ class Model:
                 if self.bad_slots_first:
                     yield ("wait", f"p_full{X % 3}", X // 3)
                 yield ("issue",)
+                if j + 2 >= d["n"]:  # this issuer's last PV of the tile
+                    yield ("commit", f"o_done{d['k'] % 2}")
                 if x is not None:
                     yield ("issue",)
                     yield ("commit", f"s_full{X % 3}")
                 yield ("commit", f"rel{(d['G0'] + j) % self.n_rel}")
+            if d["n"] == 1 and d["J0"] % 2 != me:
+                yield ("commit", f"o_done{d['k'] % 2}")
             prev = d
         yield ("commit", "drain")
         yield ("wait", "drain", 0)
@@ -182,6 +189,8 @@ class Model:
     def issuer_bad(self, me):
         """Issuer 0 alone, waiting for P_{J+1} inside group J (deadlocks on a raise)."""
         if me == 1:
+            for d in self.desc:
+                yield ("commit", f"o_done{d['k'] % 2}")
             yield ("commit", "drain")
             yield ("wait", "drain", 0)
             yield ("end",)
@@ -194,6 +203,8 @@ class Model:
             for j in range(d["n"]):
                 X = d["J0"] + j
                 yield ("issue",)
+                if j + 1 == d["n"]:
+                    yield ("commit", f"o_done{d['k'] % 2}")
                 if j + 1 < d["n"]:
                     yield ("wait", f"p_full{(X + 1) % 3}", (X + 1) // 3)
                 yield self.full(self.pos[("V", X)])
@@ -225,11 +236,9 @@ class Model:
                     if j > 1:
                         yield self.rel(d["G0"] + j - 2)
                 yield ("arrive", f"p_full{X % 3}")
-            # epilogue: every MMA of the tile has completed, then a named barrier of
-            # both groups, then the Q buffer goes back to the producer
-            yield self.rel(d["G0"] + d["n"] - 1)
-            if d["n"] >= 2:
-                yield self.rel(d["G0"] + d["n"] - 2)
+            # epilogue: every PV of the tile has completed (o_done), then a named
+            # barrier of both groups, then the Q buffer goes back to the producer
+            yield ("wait", f"o_done{d['k'] % 2}", d["k"] // 2)
             yield ("bar", u)
             if g == 0:
                 yield ("arrive", f"epi{d['k'] % 2}")
