@@ -9,12 +9,18 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/sparvar.h"
 #include "attn_fwd_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "mask_kernels.cuh"
+
+// Scratch of sparvar_block_sparse_attn_fwd_static: one array per device, in the
+// library's own module, shared by every call on that device.
+constexpr size_t kStaticScratchBytes = size_t{8} << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 namespace {
 
@@ -445,6 +451,66 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 128) return launch_attn_kernel<128, sparvar::kModeMass>(tq, tk, tk, a, st);
   return launch_attn_kernel<64, sparvar::kModeMass>(tq, tk, tk, a, st);
+}
+
+int sparvar_block_sparse_attn_fwd_static(
+    const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq,
+    int Lkv, int D, const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
+    const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
+    const int64_t* list_strides, int idx_row_len, int block, float softmax_scale,
+    int32_t* dev_status, void* stream) {
+  if (block != 16 && block != 32 && block != 64)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "block=%d not in {16, 32, 64}", block);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  if (!list_strides) return fail(SPARVAR_ERR_INVALID_ARG, "list_strides is NULL");
+  if (list_strides[0] < 0 || list_strides[1] < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
+  // tile counts, tile lists and tile masks, each 256-byte aligned, as sparvar_coarsen_lists
+  // writes them
+  const int64_t Bo = list_strides[0] == 0 ? 1 : B, Ho = list_strides[1] == 0 ? 1 : H;
+  const int64_t nqt = ceil_div(Lq, 128), nkt = ceil_div(Lkv, 128);
+  const int64_t rows = Bo * Ho * nqt;
+  auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+  const int64_t cnt_bytes = up(rows * 4), idx_bytes = up(rows * nkt * 4);
+  const int64_t need = cnt_bytes + idx_bytes + up(rows * nkt * 8);
+  if (need > static_cast<int64_t>(kStaticScratchBytes))
+    return fail(SPARVAR_ERR_UNSUPPORTED,
+                "tile lists need %lld bytes, the static scratch holds %zu",
+                static_cast<long long>(need), kStaticScratchBytes);
+  // the array's device address, looked up once per device
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return fail(SPARVAR_ERR_UNSUPPORTED, "device %d", dev);
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+      e = cudaGetSymbolAddress(&addr[dev], g_static_scratch);
+      if (e != cudaSuccess) {
+        addr[dev] = nullptr;
+        return cuda_fail(e, "cudaGetSymbolAddress");
+      }
+    }
+    base = addr[dev];
+  }
+  uint8_t* p = static_cast<uint8_t*>(base);
+  int32_t* t_cnt = reinterpret_cast<int32_t*>(p);
+  int32_t* t_idx = reinterpret_cast<int32_t*>(p + cnt_bytes);
+  uint64_t* t_mask = reinterpret_cast<uint64_t*>(p + cnt_bytes + idx_bytes);
+  int rc = sparvar_coarsen_lists(kv_cnt, kv_idx, list_strides, idx_row_len, B, H, Lq, Lkv, block,
+                                 t_cnt, t_idx, t_mask, dev_status, stream);
+  if (rc) return rc;
+  const int64_t t_strides[2] = {Bo > 1 ? Ho * nqt : 0, Ho > 1 ? nqt : 0};
+  return sparvar_block_sparse_attn_fwd(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides,
+                                       v_strides, o_strides, t_cnt, t_idx, t_strides,
+                                       static_cast<int>(nkt), t_mask, block, 128, 128,
+                                       softmax_scale, dev_status, stream);
 }
 
 }  // extern "C"

@@ -41,6 +41,9 @@ EXPORTS = {
                                        _vp], _i),
     "sparvar_map_indices_2d": ([_vp, _vp, _i, _i, _i32p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                 _vp, _vp], _i),
+    "sparvar_block_sparse_attn_fwd_static": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
+                                              _i64p, _i64p, _i64p, _vp, _vp, _i64p, _i, _i, _f,
+                                              _vp, _vp], _i),
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
@@ -197,6 +200,32 @@ def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
         _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], _ptr(tile_mask), mask_block,
         128, 128, scale, _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sparvar_block_sparse_attn_fwd_static(q, k, v, kv_cnt, kv_idx, block, softmax_scale=None,
+                                         out=None, return_lse=False, dev_status=None):
+    """Fine-grid (16/32/64) attention whose tile lists live in the library's static
+    device scratch: the only allocations here are the outputs, made by torch."""
+    B, H, Lq, D = q.shape
+    Lkv = k.shape[2]
+    if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
+        raise SparvarError("k/v must be [B, H, Lkv, D] matching q")
+    qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    os_ = _bhrd(out, "out")
+    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32:
+        raise SparvarError("kv_cnt/kv_idx must be int32")
+    if kv_idx.shape[:-1] != kv_cnt.shape or not kv_idx.is_contiguous():
+        raise SparvarError("kv_idx must be contiguous with shape (*kv_cnt.shape, row_len)")
+    lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    sb, sh = _list_strides(kv_cnt, B, H)
+    _check(lib().sparvar_block_sparse_attn_fwd_static(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
+        _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], block, scale,
+        _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd_static")
     return (out, lse) if return_lse else out
 
 

@@ -264,6 +264,34 @@ SPARVAR_API int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_i
                                       int32_t* dev_status, void* stream);
 
 /*
+ * Fine-grid attention that allocates nothing: the same result as
+ * sparvar_coarsen_lists followed by sparvar_block_sparse_attn_fwd with
+ * mask_block = block, with the tile lists and masks held in a static device
+ * array of the library (8 MiB per device, its address looked up once per
+ * device).  The pages have no counterpart; this is for callers that cannot
+ * allocate device memory.
+ *
+ * Arguments as for sparvar_block_sparse_attn_fwd, with kv_cnt/kv_idx/list_strides/
+ * idx_row_len describing lists over square blocks of side `block` (16, 32 or 64)
+ * as for sparvar_coarsen_lists.  Returns SPARVAR_ERR_UNSUPPORTED, enqueuing
+ * nothing, when the tile lists would not fit: Bo*Ho*ceil(Lq/128) rows of
+ * 4 + 12*ceil(Lkv/128) bytes (each part rounded up to 256 bytes), with Bo and Ho
+ * as for sparvar_coarsen_lists.
+ *
+ * The scratch is shared by every call on the device: calls must be ordered
+ * (one stream, or ordered by events); two calls in flight at once on different
+ * streams or host threads overwrite each other's tile lists.  Each call's
+ * coarsening writes every scratch byte its attention launch reads, so nothing
+ * must start at zero.
+ */
+SPARVAR_API int sparvar_block_sparse_attn_fwd_static(
+    const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq,
+    int Lkv, int D, const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
+    const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
+    const int64_t* list_strides, int idx_row_len, int block, float softmax_scale,
+    int32_t* dev_status, void* stream);
+
+/*
  * Device-side check of block lists: for each of n_rows rows,
  * 0 <= cnt <= min(idx_row_len, nkb), entries in [0, nkb) and strictly ascending.
  * ORs SPARVAR_DEV_BAD_LIST / SPARVAR_DEV_NOT_ASCENDING into *dev_status (required).
