@@ -440,6 +440,43 @@ def map_indices_2d(src_cnt, src_idx, sides, src_scale, dst_scale, block_q, block
 
 
 # ----------------------------------------------------------------------------
+# CS4A output cache  [M]
+# ----------------------------------------------------------------------------
+def nearest_source(i, s_src, s_dst):
+    """Row (or column) of a side-s_src grid that row i of a side-s_dst grid
+    upsamples from: floor(i * s_src / s_dst)."""
+    return (i * s_src) // s_dst
+
+
+def ocache_residual(o_dense, o_sparse):
+    """[M] CS4A keeps "the residual output left over at the decision scale" as a
+    cache.  Reading: the part of the decision scale's dense attention output that
+    its own block-sparse output (with the blocks the decision keeps) misses,
+    R = O_dense - O_sparse, per token and channel."""
+    return np.asarray(o_dense, dtype=np.float64) - np.asarray(o_sparse, dtype=np.float64)
+
+
+def ocache_upsample(r, s_src, s_dst):
+    """Nearest-neighbour 2-D upsampling of a [s_src*s_src, D] token grid to
+    [s_dst*s_dst, D]: target token (i, j) takes source token
+    (nearest_source(i), nearest_source(j))."""
+    r = np.asarray(r, dtype=np.float64)
+    out = np.empty((s_dst * s_dst, r.shape[1]))
+    for i in range(s_dst):
+        for j in range(s_dst):
+            a, b = nearest_source(i, s_src, s_dst), nearest_source(j, s_src, s_dst)
+            out[i * s_dst + j] = r[a * s_src + b]
+    return out
+
+
+def ocache_apply(o_target, o_dense, o_sparse, s_src, s_dst):
+    """[M] the cache "upsampled to correct the later sparse outputs": a later
+    scale's block-sparse output plus the upsampled decision-scale residual."""
+    return np.asarray(o_target, dtype=np.float64) + ocache_upsample(
+        ocache_residual(o_dense, o_sparse), s_src, s_dst)
+
+
+# ----------------------------------------------------------------------------
 # FLOP accounting for the kept blocks (metric definition)
 # ----------------------------------------------------------------------------
 def kept_flops(blk, nq, L, block_q, block_kv, D):

@@ -5,12 +5,14 @@ scaled-dot-product attention, element-by-element Python loops, and closed
 forms (Q = 0, constant V, one-hot V, empty rows).
 """
 import math
+import os
 
 import numpy as np
 import pytest
 import torch
 
 from oracle import sparvar_oracle as orc
+from tests.conftest import GOLDEN
 
 
 def _rand(seed, *shape):
@@ -158,3 +160,42 @@ def test_plausible_mistakes_are_caught(planted):
     P = np.exp(Sm - Sm.max(1, keepdims=True))
     bad = (P / P.sum(1, keepdims=True)) @ v
     assert np.abs(bad - ref).max() > 1e-3
+
+
+# ---------------------------------------------------------------- CS4A output cache
+def test_ocache_golden():
+    od = np.array([[1.0], [2.0], [3.0], [4.0]])
+    osp = np.array([[0.5], [2.0], [2.0], [5.0]])
+    for line in open(os.path.join(GOLDEN, "ocache_tiny.txt")):
+        if not line.startswith("side"):
+            continue
+        a, b, c = [x.strip() for x in line.split("|")]
+        s_dst = int(a.split()[1])
+        ot = np.array([[float(x)] for x in b.split()])
+        want = np.array([float(x) for x in c.split()])
+        np.testing.assert_allclose(orc.ocache_apply(ot, od, osp, 2, s_dst)[:, 0], want, atol=0)
+
+
+def test_ocache_closed_forms():
+    rng = np.random.default_rng(3)
+    # every block kept: the sparse output is the dense one, the residual is zero
+    q, k, v = rng.standard_normal((64, 16)), rng.standard_normal((100, 16)), rng.standard_normal((100, 16))
+    full = np.ones((4, 7), bool)
+    o_dense, _ = orc.masked_attention(q, k, v, full, 16, 16)
+    o_sparse, _ = orc.masked_attention(q, k, v, full, 16, 16)
+    assert np.abs(orc.ocache_residual(o_dense, o_sparse)).max() == 0.0
+    r = rng.standard_normal((36, 5))
+    # same side: identity; constant field stays constant; integer factor replicates
+    np.testing.assert_array_equal(orc.ocache_upsample(r, 6, 6), r)
+    c = np.full((36, 5), 2.5)
+    np.testing.assert_array_equal(orc.ocache_upsample(c, 6, 10), np.full((100, 5), 2.5))
+    up = orc.ocache_upsample(r, 6, 12).reshape(12, 12, 5)
+    for i in range(12):
+        for j in range(12):
+            np.testing.assert_array_equal(up[i, j], r[(i // 2) * 6 + j // 2])
+    # linear in the residual, and every source token used when upsampling
+    r2 = rng.standard_normal((36, 5))
+    np.testing.assert_allclose(orc.ocache_upsample(r + 2 * r2, 6, 9),
+                               orc.ocache_upsample(r, 6, 9) + 2 * orc.ocache_upsample(r2, 6, 9))
+    used = {orc.nearest_source(i, 32, 48) for i in range(48)}
+    assert used == set(range(32))
