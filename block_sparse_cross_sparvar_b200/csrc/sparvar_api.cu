@@ -16,6 +16,7 @@
 #include "attn_fwd_kernel.cuh"
 #include "attn_kernel.cuh"
 #include "mask_kernels.cuh"
+#include "ocache_kernel.cuh"
 
 // Scratch of sparvar_block_sparse_attn_fwd_static: one array per device, in the
 // library's own module, shared by every call on that device.
@@ -451,6 +452,45 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 128) return launch_attn_kernel<128, sparvar::kModeMass>(tq, tk, tk, a, st);
   return launch_attn_kernel<64, sparvar::kModeMass>(tq, tk, tk, a, st);
+}
+
+int sparvar_ocache_apply(const void* o_target, const void* o_dense, const void* o_sparse, void* out,
+                         int B, int H, int side_src, int side_dst, int D,
+                         const int64_t* t_strides, const int64_t* d_strides,
+                         const int64_t* s_strides, const int64_t* out_strides, void* stream) {
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (side_src < 1 || side_dst < 1 || side_src > 46340 || side_dst > 46340)
+    return fail(SPARVAR_ERR_INVALID_ARG, "sides %d, %d outside [1, 46340]", side_src, side_dst);
+  if (D < 8 || D > 1024 || D % 8 != 0)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d: a multiple of 8 in [8, 1024]", D);
+  const int n_src = side_src * side_src, n_dst = side_dst * side_dst;
+  int rc;
+  if ((rc = check_operand(o_target, t_strides, B, H, n_dst, D, "o_target"))) return rc;
+  if ((rc = check_operand(o_dense, d_strides, B, H, n_src, D, "o_dense"))) return rc;
+  if ((rc = check_operand(o_sparse, s_strides, B, H, n_src, D, "o_sparse"))) return rc;
+  if ((rc = check_operand(out, out_strides, B, H, n_dst, D, "out"))) return rc;
+  sparvar::OcacheArgs a{};
+  a.o_t = static_cast<const __nv_bfloat16*>(o_target);
+  a.o_d = static_cast<const __nv_bfloat16*>(o_dense);
+  a.o_s = static_cast<const __nv_bfloat16*>(o_sparse);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.B = B; a.H = H; a.s_src = side_src; a.s_dst = side_dst; a.D = D;
+  a.t_sb = t_strides[0]; a.t_sh = t_strides[1]; a.t_sr = t_strides[2];
+  a.d_sb = d_strides[0]; a.d_sh = d_strides[1]; a.d_sr = d_strides[2];
+  a.s_sb = s_strides[0]; a.s_sh = s_strides[1]; a.s_sr = s_strides[2];
+  a.u_sb = out_strides[0]; a.u_sh = out_strides[1]; a.u_sr = out_strides[2];
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
+  const int64_t total = static_cast<int64_t>(B) * H * n_dst * (D / 8);
+  const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), static_cast<int64_t>(sms) * 8);
+  sparvar::ocache_apply_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "ocache_apply_kernel launch");
+  return SPARVAR_OK;
 }
 
 int sparvar_block_sparse_attn_fwd_static(

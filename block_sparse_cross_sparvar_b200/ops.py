@@ -44,6 +44,8 @@ EXPORTS = {
     "sparvar_block_sparse_attn_fwd_static": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
                                               _i64p, _i64p, _i64p, _vp, _vp, _i64p, _i, _i, _f,
                                               _vp, _vp], _i),
+    "sparvar_ocache_apply": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p, _i64p, _i64p,
+                              _vp], _i),
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
@@ -227,6 +229,21 @@ def sparvar_block_sparse_attn_fwd_static(q, k, v, kv_cnt, kv_idx, block, softmax
         _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], block, scale,
         _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd_static")
     return (out, lse) if return_lse else out
+
+
+def sparvar_ocache_apply(o_target, o_dense, o_sparse, side_src, side_dst, out=None):
+    """CS4A output cache: o_target + nearest-upsampled (o_dense - o_sparse)."""
+    B, H, n_dst, D = o_target.shape
+    if n_dst != side_dst * side_dst or o_dense.shape != (B, H, side_src * side_src, D) \
+            or o_sparse.shape != o_dense.shape:
+        raise SparvarError("o_target [B, H, side_dst^2, D]; o_dense, o_sparse [B, H, side_src^2, D]")
+    if out is None:
+        out = torch.empty_like(o_target, memory_format=torch.contiguous_format)
+    _check(lib().sparvar_ocache_apply(
+        _ptr(o_target), _ptr(o_dense), _ptr(o_sparse), _ptr(out), B, H, side_src, side_dst, D,
+        _bhrd(o_target, "o_target"), _bhrd(o_dense, "o_dense"), _bhrd(o_sparse, "o_sparse"),
+        _bhrd(out, "out"), _stream(o_target.device)), "sparvar_ocache_apply")
+    return out
 
 
 def sparvar_decide_blocks(q, k, mass_threshold, lse=None, softmax_scale=None, block_q=128,

@@ -264,6 +264,31 @@ SPARVAR_API int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_i
                                       int32_t* dev_status, void* stream);
 
 /*
+ * CS4A output cache ("Methodology in Plain English", CS4A paragraph: the residual
+ * output left at the decision scale is cached and upsampled to correct the
+ * later sparse outputs; "Main Findings": O_cache adds about 0.7 PSNR):
+ *
+ *   out[t] = o_target[t] + o_dense[src(t)] - o_sparse[src(t)],
+ *
+ * for target token t = (i, j) of the side-side_dst scale and src(t) the token
+ * (floor(i*side_src/side_dst), floor(j*side_src/side_dst)) of the side-side_src
+ * decision scale (nearest-neighbour upsampling); o_dense and o_sparse are the
+ * decision scale's dense output and its block-sparse output with the lists the
+ * decision keeps.  Computed in fp32 from the bf16 inputs, rounded to bf16.
+ *
+ * o_target, out [B][H][side_dst^2][D]; o_dense, o_sparse [B][H][side_src^2][D]: device
+ *   bf16 with element strides for (b, h, row) from host arrays *_strides[3]; last dim
+ *   contiguous; base addresses and strides 16-byte aligned.  D a multiple of 8 in
+ *   [8, 1024].  out may be o_target (in place); it must not overlap the other inputs.
+ */
+SPARVAR_API int sparvar_ocache_apply(const void* o_target, const void* o_dense,
+                                     const void* o_sparse, void* out, int B, int H,
+                                     int side_src, int side_dst, int D,
+                                     const int64_t* t_strides, const int64_t* d_strides,
+                                     const int64_t* s_strides, const int64_t* out_strides,
+                                     void* stream);
+
+/*
  * Fine-grid attention that allocates nothing: the same result as
  * sparvar_coarsen_lists followed by sparvar_block_sparse_attn_fwd with
  * mask_block = block, with the tile lists and masks held in a static device

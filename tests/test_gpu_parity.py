@@ -511,3 +511,61 @@ def test_cs4a_topk_2d_pipeline_attention():
         oc, oi, _ = orc.map_indices_2d(dcn[0, h], din[0, h], INF, s, t, 128, 128, off[5])
         assert np.array_equal(mc[0, h].cpu().numpy(), oc)
         assert np.array_equal(mi[0, h].cpu().numpy(), oi)
+
+
+# ------------------------------------------------------------------ CS4A output cache
+@pytest.mark.parametrize("s_src,s_dst,D", [(32, 64, 128), (32, 40, 128), (32, 48, 64), (7, 7, 128),
+                                           (5, 13, 64)])
+def test_ocache_apply_elementwise(s_src, s_dst, D):
+    rng = np.random.default_rng(s_src * s_dst + D)
+    B, H = 2, 3
+    mk = lambda n: inputs.bf16_round(rng.standard_normal((B, H, n, D)).astype(np.float32))[0]  # noqa: E731
+    t_bits, d_bits, s_bits = mk(s_dst * s_dst), mk(s_src * s_src), mk(s_src * s_src)
+    t_dev = _dev(t_bits)
+    # strided view for the target: every other head of a wider tensor
+    wide = torch.zeros(B, 2 * H, s_dst * s_dst, D, dtype=torch.bfloat16, device="cuda")
+    wide[:, ::2] = t_dev
+    out = ops.sparvar_ocache_apply(wide[:, ::2], _dev(d_bits), _dev(s_bits), s_src, s_dst)
+    inplace = t_dev.clone()
+    ops.sparvar_ocache_apply(inplace, _dev(d_bits), _dev(s_bits), s_src, s_dst, out=inplace)
+    torch.cuda.synchronize()
+    assert torch.equal(out, inplace)
+    got = out.float().cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            want = orc.ocache_apply(q_bits_f(t_bits, b, h), q_bits_f(d_bits, b, h),
+                                    q_bits_f(s_bits, b, h), s_src, s_dst)
+            assert np.all(np.abs(got[b, h] - want) <= np.abs(want) * 2.0 ** -8 + 1e-6)
+
+
+def test_cs4a_with_ocache_pipeline():
+    """Decision at 32x32, the decision scale's sparse output, mapping to 40x40, the
+    sparse output there corrected by the cache, against the oracle chain in fp64."""
+    d = inputs.make_qkv(12, 1, 2, INF, 128, 5)
+    off = d["offsets"]
+    s, t = 9, 10
+    qd, kd, vd = d["q"][:, :, off[s]:off[s + 1]], d["k"][:, :, :off[s + 1]], d["v"][:, :, :off[s + 1]]
+    nqb, nkb = 8, -(-off[s + 1] // 128)
+    dense_c = torch.full((nqb,), nkb, dtype=torch.int32, device="cuda")
+    dense_i = torch.arange(nkb, dtype=torch.int32, device="cuda").repeat(nqb, 1).contiguous()
+    o_dense, lse = ops.sparvar_block_sparse_attn_fwd(_dev(qd), _dev(kd), _dev(vd), dense_c, dense_i,
+                                                     return_lse=True)
+    dc, di, _ = ops.sparvar_decide_blocks(_dev(qd), _dev(kd), 0.0, lse=lse, topk_ratio=0.2)
+    o_sparse = ops.sparvar_block_sparse_attn_fwd(_dev(qd), _dev(kd), _dev(vd), dc, di)
+    qt, kt, vt = d["q"][:, :, off[t]:off[t + 1]], d["k"][:, :, :off[t + 1]], d["v"][:, :, :off[t + 1]]
+    mc, mi, _ = ops.sparvar_map_indices(dc, di, 1024, off[s + 1], 1600, off[t + 1], 128, 128, off[5])
+    o_t = ops.sparvar_block_sparse_attn_fwd(_dev(qt), _dev(kt), _dev(vt), mc, mi)
+    out = ops.sparvar_ocache_apply(o_t, o_dense, o_sparse, INF[s], INF[t])
+    torch.cuda.synchronize()
+    dcn, din, mcn, min_ = dc.cpu().numpy(), di.cpu().numpy(), mc.cpu().numpy(), mi.cpu().numpy()
+    for h in range(2):
+        Od, _ = orc.masked_attention(q_bits_f(qd, 0, h), q_bits_f(kd, 0, h), q_bits_f(vd, 0, h),
+                                     np.ones((nqb, nkb), bool), 128, 128)
+        Os, _ = orc.masked_attention(q_bits_f(qd, 0, h), q_bits_f(kd, 0, h), q_bits_f(vd, 0, h),
+                                     orc.lists_to_blocks(dcn[0, h], din[0, h], nkb), 128, 128)
+        Ot, _ = orc.masked_attention(q_bits_f(qt, 0, h), q_bits_f(kt, 0, h), q_bits_f(vt, 0, h),
+                                     orc.lists_to_blocks(mcn[0, h], min_[0, h], -(-off[t + 1] // 128)),
+                                     128, 128)
+        want = orc.ocache_apply(Ot, Od, Os, INF[s], INF[t])
+        err = np.abs(out[0, h].float().cpu().numpy() - want)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())

@@ -141,3 +141,18 @@ def test_map_2d_rejects_bad_arguments(lib):
     assert call(bq=8) == 2
     assert call(sink=-1) == 1
     assert call(cnt=0) == 1
+
+
+def test_ocache_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    i64 = lambda *x: (ctypes.c_int64 * len(x))(*x)  # noqa: E731
+    st = i64(0, 0, 128)
+
+    def call(D=128, s_src=32, s_dst=64, ot=16, od=16):
+        return lib.sparvar_ocache_apply(vp(ot), vp(od), vp(16), vp(16), 1, 1, s_src, s_dst, D, st, st,
+                                        st, st, vp(0))
+
+    assert call(D=12) == 2 and "D=12" in lib.sparvar_last_error().decode()
+    assert call(s_src=0) == 1
+    assert call(ot=0) == 1 and "o_target" in lib.sparvar_last_error().decode()
+    assert call(od=8) == 1 and "aligned" in lib.sparvar_last_error().decode()
