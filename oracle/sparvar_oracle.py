@@ -171,6 +171,26 @@ def masked_attention(q, k, v, blk, block_q, block_kv, scale=None, return_p=False
     return O, lse
 
 
+def masked_attention_tokens(q, k, v, token_mask, scale=None):
+    """O = softmax(scale * q k^T, -inf where token_mask is False) v, in fp64: the
+    CSLA token mask applied exactly instead of through its blocks.  Rows whose
+    every key is masked give O = 0 and LSE = -inf.  Returns (O, lse)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[1])
+    S = np.where(token_mask, scale * (q @ k.T), -np.inf)
+    m = S.max(axis=1)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    P = np.exp(S - m_safe[:, None])
+    l = P.sum(axis=1)
+    l_safe = np.where(empty, 1.0, l)
+    O = (P / l_safe[:, None]) @ v
+    return O, np.where(empty, -np.inf, m_safe + np.log(l_safe))
+
+
 def masked_attention_rows(rows, q, k, v, blk, block_q, block_kv, scale=None):
     """The same definition evaluated for selected query rows only."""
     rows = np.asarray(rows)

@@ -199,3 +199,43 @@ def test_ocache_closed_forms():
                                orc.ocache_upsample(r, 6, 9) + 2 * orc.ocache_upsample(r2, 6, 9))
     used = {orc.nearest_source(i, 32, 48) for i in range(48)}
     assert used == set(range(32))
+
+
+# ---------------------------------------------------------------- token-level masks
+def test_token_mask_attention_pins():
+    rng = np.random.default_rng(21)
+    q, k, v = rng.standard_normal((40, 8)), rng.standard_normal((70, 8)), rng.standard_normal((70, 8))
+    # a block-structured token mask gives the block function's result
+    blk = rng.random((3, 5)) < 0.5
+    blk[:, 0] = True
+    E = orc.expand_block_mask(blk, 40, 70, 16, 16)
+    O1, L1 = orc.masked_attention_tokens(q, k, v, E)
+    O2, L2 = orc.masked_attention(q, k, v, blk, 16, 16)
+    np.testing.assert_allclose(O1, O2, atol=1e-14)
+    np.testing.assert_allclose(L1, L2, atol=1e-14)
+    # brute force on a random token mask, element by element
+    T = rng.random((40, 70)) < 0.3
+    T[5] = False  # an empty row
+    O, lse = orc.masked_attention_tokens(q, k, v, T, scale=0.4)
+    for i in range(40):
+        keys = np.nonzero(T[i])[0]
+        if keys.size == 0:
+            assert np.all(O[i] == 0) and lse[i] == -np.inf
+            continue
+        s = [0.4 * sum(q[i, d] * k[j, d] for d in range(8)) for j in keys]
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        z = sum(w)
+        for d in range(8):
+            assert abs(O[i, d] - sum(w[t] * v[j, d] for t, j in enumerate(keys)) / z) < 1e-12
+        assert abs(lse[i] - (mx + math.log(z))) < 1e-12
+
+
+def test_csla_token_mask_inside_its_blocks():
+    # the CSLA block mask is the token mask's aggregate, so masking by tokens inside the
+    # kept blocks is masking by tokens
+    sides = (1, 2, 4, 8, 16)
+    T = orc.csla_token_mask(sides, 4, 2, 1, 1)
+    cnt, idx, blk = orc.build_csla_mask(sides, 4, 2, 1, 1, 16, 16)
+    E = orc.expand_block_mask(blk, T.shape[0], T.shape[1], 16, 16)
+    assert np.all(E[T]) and (E & ~T).any()
