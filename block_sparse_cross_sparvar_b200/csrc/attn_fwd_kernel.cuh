@@ -73,6 +73,15 @@ constexpr int kRel = 16;                      // release barriers (more than rin
 // (exp2_poly2), the others the MUFU ex2.
 constexpr uint32_t kPolyPairs = 0x0u;
 
+// CSLA token mask applied inside the kept tiles (enabled != 0): the query scale,
+// the sink length in tokens and the locality radii over the schedule.
+struct CslaTokens {
+  int enabled;
+  int q_scale, n_sink_scales, n_sink_tok, r_prev, r_own;
+  int side[32];
+  int off[33];
+};
+
 struct Args {
   int B, H, Lq, Lkv, nqb, nkb;
   float scale_log2;  // softmax_scale * log2(e)
@@ -86,6 +95,7 @@ struct Args {
   int64_t o_sb, o_sh, o_sr;
   float* lse;  // [B][H][Lq] or null
   int32_t* dev_status;
+  CslaTokens tok;
 };
 
 struct __align__(8) Bars {
@@ -208,13 +218,51 @@ __device__ __forceinline__ bool warp_wait_group(uint64_t* rel, int grp, volatile
   return warp_wait(&rel[grp % kRel], (grp / kRel) & 1, abort, st);
 }
 
+// OR columns [lo, hi) (0 <= lo < hi <= 128) into a 128-bit row mask
+__device__ __forceinline__ void set_cols(uint32_t (&km)[4], int lo, int hi) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int a = max(lo, w * 32), b = min(hi, w * 32 + 32);
+    if (a < b) km[w] |= (b - a == 32 ? 0xffffffffu : ((1u << (b - a)) - 1u)) << (a - w * 32);
+  }
+}
+
+// CSLA token mask of query (i, j) of the query scale over keys [k0, k1): the sink,
+// and for every scale m from the first non-sink one up to the query scale, the keys
+// within Chebyshev radius r_m of the query's projection (floor(i*s_m/s_k),
+// floor(j*s_m/s_k)); the rows of that window meeting [k0, k1) are contiguous
+// column ranges.
+__device__ __forceinline__ void csla_row_mask(const CslaTokens& t, int i, int j, int k0, int k1,
+                                              uint32_t (&km)[4]) {
+  km[0] = km[1] = km[2] = km[3] = 0u;
+  if (k0 < t.n_sink_tok) set_cols(km, 0, min(t.n_sink_tok, k1) - k0);
+  const int sk = t.side[t.q_scale];
+  for (int m = t.n_sink_scales; m <= t.q_scale; ++m) {
+    const int o0 = t.off[m], o1 = t.off[m + 1];
+    if (o1 <= k0 || o0 >= k1) continue;
+    const int sm = t.side[m];
+    const int r = m == t.q_scale ? t.r_own : t.r_prev;
+    const int ci = static_cast<int>(static_cast<int64_t>(i) * sm / sk);
+    const int cj = static_cast<int>(static_cast<int64_t>(j) * sm / sk);
+    const int c0 = max(cj - r, 0), c1 = min(cj + r, sm - 1);
+    const int a0 = max(max(ci - r, 0), (max(k0, o0) - o0) / sm);
+    const int a1 = min(min(ci + r, sm - 1), (min(k1, o1) - 1 - o0) / sm);
+    for (int a = a0; a <= a1; ++a) {
+      const int lo = max(o0 + a * sm + c0, k0) - k0;
+      const int hi = min(o0 + a * sm + c1 + 1, k1) - k0;
+      if (lo < hi) set_cols(km, lo, hi);
+    }
+  }
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
-template <int D>
+// TOK: apply the CSLA token mask (args.tok) inside the kept tiles
+template <int D, bool TOK>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -447,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (TileCursor c = first; c.t < total; cursor_next(c, args, total, threadIdx.x == 0)) {
       float m_own = -INFINITY;  // reference of this group's row sum
       float l_own = 0.f;
+      const int c_qb = TOK ? c.t % args.nqb : 0;
       for (int j = ((c.J0 & 1) == g) ? 0 : 1; j < c.n && good; j += 2) {
         const int J = c.J0 + j;
         const int kb = __ldg(c.list + j);
@@ -476,8 +525,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           fine = __any_sync(0xffffffffu, keep != full);
           keep |= ~full;
         }
+        // with the CSLA token mask on, bit c of km keeps column c of this row
+        uint32_t km[4] = {~0u, ~0u, ~0u, ~0u};
+        if constexpr (TOK) {
+          const int grow = c_qb * kTile + row;
+          const int sk = args.tok.side[args.tok.q_scale];
+          const int gq = grow < args.Lq ? grow : 0;
+          if (valid > 0)
+            csla_row_mask(args.tok, gq / sk, gq % sk, kb * kTile, kb * kTile + valid, km);
+          fine = true;
+        }
         auto dropped = [&](int col) {
-          return col >= valid || !((keep >> (col >> args.mask_shift)) & 1u);
+          return col >= valid || !((keep >> (col >> args.mask_shift)) & 1u) ||
+                 !((km[col >> 5] >> (col & 31)) & 1u);
         };
         // pass 1: the block's row max.  Columns 0-95 stay in registers for pass 2.
         float bm;

@@ -139,10 +139,10 @@ int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   return SPARVAR_OK;
 }
 
-template <int D>
+template <int D, bool TOK>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const sparvar::fwd::Args& a, cudaStream_t stream) {
-  auto kern = sparvar::fwd::attn_fwd_kernel<D>;
+  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -342,15 +342,14 @@ int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_r
   return SPARVAR_OK;
 }
 
-int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
-                                  float* lse, int B, int H, int Lq, int Lkv, int D,
-                                  const int64_t* q_strides, const int64_t* k_strides,
-                                  const int64_t* v_strides, const int64_t* o_strides,
-                                  const int32_t* kv_cnt, const int32_t* kv_idx,
-                                  const int64_t* list_strides, int idx_row_len,
-                                  const uint64_t* tile_mask, int mask_block, int block_q,
-                                  int block_kv, float softmax_scale, int32_t* dev_status,
-                                  void* stream) {
+static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Lq, int Lkv, int D, const int64_t* q_strides,
+                         const int64_t* k_strides, const int64_t* v_strides,
+                         const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
+                         const int64_t* list_strides, int idx_row_len, const uint64_t* tile_mask,
+                         int mask_block, int block_q, int block_kv, float softmax_scale,
+                         int32_t* dev_status, void* stream,
+                         const sparvar::fwd::CslaTokens* tok) {
   if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
   if (block_q != 128 || block_kv != 128)
     return fail(SPARVAR_ERR_UNSUPPORTED,
@@ -395,6 +394,7 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
   a.lse = lse;
   a.dev_status = dev_status;
+  if (tok) a.tok = *tok;
 
   CUtensorMap tq, tk, tv, to;
   if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
@@ -402,8 +402,56 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
   if ((rc = make_tmap(&to, o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o"))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_fwd_kernel<128>(tq, tk, tv, to, a, st);
-  return launch_fwd_kernel<64>(tq, tk, tv, to, a, st);
+  if (tok) {
+    if (D == 128) return launch_fwd_kernel<128, true>(tq, tk, tv, to, a, st);
+    return launch_fwd_kernel<64, true>(tq, tk, tv, to, a, st);
+  }
+  if (D == 128) return launch_fwd_kernel<128, false>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64, false>(tq, tk, tv, to, a, st);
+}
+
+int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int H, int Lq, int Lkv, int D,
+                                  const int64_t* q_strides, const int64_t* k_strides,
+                                  const int64_t* v_strides, const int64_t* o_strides,
+                                  const int32_t* kv_cnt, const int32_t* kv_idx,
+                                  const int64_t* list_strides, int idx_row_len,
+                                  const uint64_t* tile_mask, int mask_block, int block_q,
+                                  int block_kv, float softmax_scale, int32_t* dev_status,
+                                  void* stream) {
+  return attn_fwd_impl(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides, v_strides,
+                       o_strides, kv_cnt, kv_idx, list_strides, idx_row_len, tile_mask, mask_block,
+                       block_q, block_kv, softmax_scale, dev_status, stream, nullptr);
+}
+
+int sparvar_csla_token_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int D, const int64_t* q_strides,
+                                const int64_t* k_strides, const int64_t* v_strides,
+                                const int64_t* o_strides, const int32_t* sides, int n_scales,
+                                int q_scale, int n_sink_scales, int radius_prev, int radius_own,
+                                const int32_t* kv_cnt, const int32_t* kv_idx,
+                                const int64_t* list_strides, int idx_row_len,
+                                float softmax_scale, int32_t* dev_status, void* stream) {
+  sparvar::ScaleGeometry g;
+  int rc = build_geometry(sides, n_scales, &g);
+  if (rc) return rc;
+  if (q_scale < 0 || q_scale >= n_scales)
+    return fail(SPARVAR_ERR_INVALID_ARG, "q_scale=%d outside [0, %d)", q_scale, n_scales);
+  if (n_sink_scales < 0 || radius_prev < 0 || radius_own < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "n_sink_scales and radii must be >= 0");
+  sparvar::fwd::CslaTokens t{};
+  t.enabled = 1;
+  t.q_scale = q_scale;
+  t.n_sink_scales = n_sink_scales;
+  t.n_sink_tok = g.off[std::min(n_sink_scales, q_scale + 1)];
+  t.r_prev = radius_prev;
+  t.r_own = radius_own;
+  for (int m = 0; m < n_scales; ++m) t.side[m] = g.side[m];
+  for (int m = 0; m <= n_scales; ++m) t.off[m] = g.off[m];
+  const int Lq = g.side[q_scale] * g.side[q_scale], Lkv = g.off[q_scale + 1];
+  return attn_fwd_impl(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides, v_strides,
+                       o_strides, kv_cnt, kv_idx, list_strides, idx_row_len, nullptr, 0, 128, 128,
+                       softmax_scale, dev_status, stream, &t);
 }
 
 int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, int Lkv, int D,

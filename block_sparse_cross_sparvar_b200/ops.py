@@ -46,6 +46,9 @@ EXPORTS = {
                                               _vp, _vp], _i),
     "sparvar_ocache_apply": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p, _i64p, _i64p,
                               _vp], _i),
+    "sparvar_csla_token_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i64p, _i64p, _i64p,
+                                     _i64p, _i32p, _i, _i, _i, _i, _i, _vp, _vp, _i64p, _i, _f,
+                                     _vp, _vp], _i),
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
@@ -228,6 +231,34 @@ def sparvar_block_sparse_attn_fwd_static(q, k, v, kv_cnt, kv_idx, block, softmax
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
         _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], block, scale,
         _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd_static")
+    return (out, lse) if return_lse else out
+
+
+def sparvar_csla_token_attn_fwd(q, k, v, sides, q_scale, n_sink_scales, radius_prev, radius_own,
+                                kv_cnt, kv_idx, softmax_scale=None, out=None, return_lse=False,
+                                dev_status=None):
+    """Attention under the CSLA token mask inside the listed 128x128 tiles."""
+    B, H, Lq, D = q.shape
+    Lkv = k.shape[2]
+    off = [0]
+    for s_ in sides:
+        off.append(off[-1] + s_ * s_)
+    if Lq != sides[q_scale] ** 2 or Lkv != off[q_scale + 1]:
+        raise SparvarError("q must hold the query scale's tokens and k/v its prefix")
+    qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32 or not kv_idx.is_contiguous():
+        raise SparvarError("kv_cnt/kv_idx must be int32, kv_idx contiguous")
+    lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    sb, sh = _list_strides(kv_cnt, B, H)
+    arr = (ctypes.c_int32 * len(sides))(*sides)
+    _check(lib().sparvar_csla_token_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, D, qs, ks, vs, _bhrd(out, "out"), arr,
+        len(sides), q_scale, n_sink_scales, radius_prev, radius_own, _ptr(kv_cnt), _ptr(kv_idx),
+        _i64([sb, sh]), kv_idx.shape[-1], scale, _ptr(dev_status), _stream(q.device)),
+        "sparvar_csla_token_attn_fwd")
     return (out, lse) if return_lse else out
 
 

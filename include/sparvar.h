@@ -264,6 +264,31 @@ SPARVAR_API int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_i
                                       int32_t* dev_status, void* stream);
 
 /*
+ * Block-sparse attention with the CSLA token mask applied inside the kept tiles
+ * ("Methodology in Plain English", CSLA paragraph: the token-wise mask, here used
+ * as it is rather than only through its blocks): O[q] = sum_key softmax(s(q,key)) V[key] over the keys the CSLA token
+ * rule of sparvar_build_csla_mask keeps for q, taken from the listed 128x128
+ * tiles (pass the lists sparvar_build_csla_mask writes at block 128; a key the
+ * rule keeps outside the listed tiles does not contribute).
+ *
+ * Geometry (host sides[n_scales], q_scale, n_sink_scales, radius_prev,
+ * radius_own) as for sparvar_build_csla_mask; Lq = sides[q_scale]^2 and Lkv =
+ * the prefix length through q_scale.  q, k, v, o, lse, the lists, the scale and
+ * dev_status as for sparvar_block_sparse_attn_fwd (D in {64, 128}).  A query
+ * whose kept keys all fall outside the listed tiles gets O = 0, lse = -inf.
+ */
+SPARVAR_API int sparvar_csla_token_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                            float* lse, int B, int H, int D,
+                                            const int64_t* q_strides, const int64_t* k_strides,
+                                            const int64_t* v_strides, const int64_t* o_strides,
+                                            const int32_t* sides, int n_scales, int q_scale,
+                                            int n_sink_scales, int radius_prev, int radius_own,
+                                            const int32_t* kv_cnt, const int32_t* kv_idx,
+                                            const int64_t* list_strides, int idx_row_len,
+                                            float softmax_scale, int32_t* dev_status,
+                                            void* stream);
+
+/*
  * CS4A output cache ("Methodology in Plain English", CS4A paragraph: the residual
  * output left at the decision scale is cached and upsampled to correct the
  * later sparse outputs; "Main Findings": O_cache adds about 0.7 PSNR):

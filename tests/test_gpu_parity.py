@@ -569,3 +569,49 @@ def test_cs4a_with_ocache_pipeline():
         want = orc.ocache_apply(Ot, Od, Os, INF[s], INF[t])
         err = np.abs(out[0, h].float().cpu().numpy() - want)
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+
+
+# ------------------------------------------------------------------ CSLA token mask
+def _token_check(sides, q_scale, ns, rp, ro, B, H, D, seed, rows=None, pe=True):
+    d = inputs.make_qkv(seed, B, H, sides, D, ns, pe=pe)
+    off = d["offsets"]
+    q_bits = d["q"][:, :, off[q_scale]:off[q_scale + 1]]
+    L = off[q_scale + 1]
+    cnt, idx, _ = ops.sparvar_build_csla_mask(sides, q_scale, ns, rp, ro, 128, 128)
+    st = _status()
+    o, lse = ops.sparvar_csla_token_attn_fwd(_dev(q_bits), _dev(d["k"][:, :, :L]),
+                                             _dev(d["v"][:, :, :L]), sides, q_scale, ns, rp, ro,
+                                             cnt, idx, return_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    T = orc.csla_token_mask(sides, q_scale, ns, rp, ro)
+    if rows is None:
+        rows = np.arange(T.shape[0])
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            O, Lo = orc.masked_attention_tokens(q_bits_f(q_bits, b, h)[rows], q_bits_f(d["k"][:, :, :L], b, h),
+                                                q_bits_f(d["v"][:, :, :L], b, h), T[rows])
+            err = np.abs(o[b, h, rows] - O)
+            assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (b, h, err.max(), err.mean())
+            assert np.abs(lse[b, h, rows] - Lo).max() < 1e-3
+    # the token mask drops keys the block path keeps: the outputs differ
+    o_blk = ops.sparvar_block_sparse_attn_fwd(_dev(q_bits), _dev(d["k"][:, :, :L]),
+                                              _dev(d["v"][:, :, :L]), cnt, idx).float().cpu().numpy()
+    assert np.abs(o_blk - o).max() > 1e-3
+
+
+@pytest.mark.parametrize("q_scale,D", [(3, 64), (4, 64), (4, 128)])
+def test_csla_token_attention_tiny(q_scale, D):
+    _token_check(TINY, q_scale, 2, 1, 1, 1, 2, D, 31 + q_scale, pe=False)
+
+
+@pytest.mark.parametrize("q_scale,rp", [(9, 2), (10, 1), (11, 4)])
+def test_csla_token_attention_infinity(q_scale, rp):
+    _token_check(INF, q_scale, 5, rp, 4, 1, 2, 128, q_scale)
+
+
+def test_csla_token_attention_last_scale_sampled_rows():
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([rng.integers(0, 4096, 48), [0, 63, 64, 4095]]))
+    _token_check(INF, 12, 5, 2, 4, 2, 2, 128, 7, rows=rows)
