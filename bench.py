@@ -346,7 +346,7 @@ def main():
             from block_sparse_cross_sparvar_b200 import workloads
             del q, kk, vv, o, hq, hk, hv
             torch.cuda.empty_cache()
-            for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass,
+            for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass, workloads.cs4a_fused_pass,
                        workloads.csla_radius_sweep, workloads.density_sweep):
                 print(json.dumps({"extra": fn(dev)}), flush=True)
                 torch.cuda.empty_cache()

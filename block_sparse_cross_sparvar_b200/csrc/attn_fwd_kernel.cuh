@@ -82,20 +82,38 @@ struct CslaTokens {
   int off[33];
 };
 
-struct Args {
-  int B, H, Lq, Lkv, nqb, nkb;
-  float scale_log2;  // softmax_scale * log2(e)
+// One attention problem of a launch: queries [q_row0, q_row0 + Lq) of the Q, O
+// and LSE row space attend to keys [0, Lkv) under their own block lists.  A
+// launch walks the tiles of all its problems (one problem unless several
+// scales share a launch).
+constexpr int kMaxProblems = 16;
+struct Problem {
+  int Lq, Lkv, nqb, nkb;
+  int q_row0;
+  int tile0;  // first tile id of the problem in the launch
+  int idx_row_len;
   const int32_t* kv_cnt;
   const int32_t* kv_idx;
   int64_t list_sb, list_sh;
-  int idx_row_len;
+};
+
+struct Args {
+  int B, H, n_problems, total_tiles;
+  float scale_log2;  // softmax_scale * log2(e)
+  Problem prob[kMaxProblems];
   const uint64_t* tile_mask;  // per list entry, fine-block bits; null: whole tiles
   int mask_shift;             // log2 of the fine block side (4, 5 or 6)
   __nv_bfloat16* o;
   int64_t o_sb, o_sh, o_sr;
-  float* lse;  // [B][H][Lq] or null
+  float* lse;    // [B][H][lse_rows] or null
+  int lse_rows;
   int32_t* dev_status;
   CslaTokens tok;
+};
+
+// output tensor map of each problem (its rows only, so ragged tiles are clipped)
+struct OutMaps {
+  CUtensorMap m[kMaxProblems];
 };
 
 struct __align__(8) Bars {
@@ -126,7 +144,8 @@ struct Layout {
 // stream.  Any other non-empty tile starts with a prologue group (its first
 // score MMAs, issued once the predecessor's MMAs are done).
 struct TileCursor {
-  int t;  // tile id (b * H + h) * nqb + qb; >= total when the CTA is done
+  int t;  // tile id (problem tile0 + (b * H + h) * nqb + qb); >= total when the CTA is done
+  int p;  // problem of the tile
   int n;  // list length (clamped to [0, idx_row_len])
   const int32_t* list;
   int J0;      // sequence index of the tile's first block
@@ -138,32 +157,43 @@ struct TileCursor {
 };
 
 struct TileCoord {
-  int b, h, qb;
+  int p, b, h, qb;
 };
+template <bool MULTI>
 __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
-  const int bh = t / a.nqb;
-  return TileCoord{bh / a.H, bh % a.H, t % a.nqb};
+  int p = 0;
+  if constexpr (MULTI) {
+    while (p + 1 < a.n_problems && t >= a.prob[p + 1].tile0) ++p;
+  }
+  const Problem& pr = a.prob[p];
+  const int lt = t - pr.tile0;
+  const int bh = lt / pr.nqb;
+  return TileCoord{p, bh / a.H, bh % a.H, lt % pr.nqb};
 }
 
+template <bool MULTI>
 __device__ __forceinline__ int tile_count(int t, const Args& a, bool report,
-                                          const int32_t** list) {
-  const TileCoord tc = tile_coord(t, a);
-  const int64_t lrow = tc.b * a.list_sb + tc.h * a.list_sh + tc.qb;
-  int n = __ldg(a.kv_cnt + lrow);
-  if (n < 0 || n > a.idx_row_len) {
+                                          const int32_t** list, int* prob) {
+  const TileCoord tc = tile_coord<MULTI>(t, a);
+  const Problem& pr = a.prob[tc.p];
+  const int64_t lrow = tc.b * pr.list_sb + tc.h * pr.list_sh + tc.qb;
+  int n = __ldg(pr.kv_cnt + lrow);
+  if (n < 0 || n > pr.idx_row_len) {
     if (report && a.dev_status) atomicOr(a.dev_status, 0x1);
-    n = n < 0 ? 0 : a.idx_row_len;
+    n = n < 0 ? 0 : pr.idx_row_len;
   }
-  if (list) *list = a.kv_idx + lrow * a.idx_row_len;
+  if (list) *list = pr.kv_idx + lrow * pr.idx_row_len;
+  if (prob) *prob = tc.p;
   return n;
 }
 
+template <bool MULTI>
 __device__ __forceinline__ void cursor_load(TileCursor& c, const Args& a, int total, bool report) {
   if (c.t >= total) return;
-  c.n = tile_count(c.t, a, report, &c.list);
+  c.n = tile_count<MULTI>(c.t, a, report, &c.list, &c.p);
   c.next_n = 0;
   for (int t = c.t + gridDim.x; t < total && c.next_n == 0; t += gridDim.x)
-    c.next_n = tile_count(t, a, false, nullptr);
+    c.next_n = tile_count<MULTI>(t, a, false, nullptr, nullptr);
 }
 
 __device__ __forceinline__ bool has_prologue(const TileCursor& c) { return c.prev_n < 3; }
@@ -192,6 +222,7 @@ __device__ __forceinline__ int group_of_block(const TileCursor& c, int j) {
   return c.G + (has_prologue(c) ? 1 : 0) + j;
 }
 
+template <bool MULTI>
 __device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int total, bool report) {
   if (c.n > 0) {
     c.pos0 += ring_items(c);
@@ -201,7 +232,7 @@ __device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int to
     c.prev_n = c.n;
   }
   c.t += gridDim.x;
-  cursor_load(c, a, total, report);
+  cursor_load<MULTI>(c, a, total, report);
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -261,13 +292,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// TOK: apply the CSLA token mask (args.tok) inside the kept tiles
-template <int D, bool TOK>
+// TOK: apply the CSLA token mask (args.tok) inside the kept tiles.  MULTI: the
+// launch holds several problems (args.prob), one output map each.
+template <int D, bool TOK, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Args args) {
+                    const __grid_constant__ OutMaps tm_os, const __grid_constant__ Args args) {
   using L = Layout<D>;
   constexpr int NS = L::kSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -283,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
   volatile int* abort_flag = &abort_sh;
   int32_t* dev_status = args.dev_status;
-  const int total = args.B * args.H * args.nqb;
+  const int total = args.total_tiles;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -311,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_o);
+    prefetch_tmap(&tm_os.m[0]);
   }
   tc_fence_before();
   __syncthreads();
@@ -323,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileCursor first{};
   first.t = blockIdx.x;
   first.prev_n = -1;
-  cursor_load(first, args, total, threadIdx.x == 0);
+  cursor_load<MULTI>(first, args, total, threadIdx.x == 0);
 
   if (warp == kLoadWarp) {
     // ================================================================ producer
@@ -339,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           return;
         }
         relg_sh[s] = grp;
-        kb = kb < 0 ? -1 : (kb > args.nkb ? args.nkb : kb);
+        const int nkb_p = args.prob[tc.p].nkb;
+        kb = kb < 0 ? -1 : (kb > nkb_p ? nkb_p : kb);
         mbar_arrive_expect_tx(&bars.full[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
@@ -359,12 +392,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < L::kChunks; ++cc)
           tma_load_4d(sQ(k) + cc * L::kChunkBytes, &tm_q, &bars.q_full[qs], cc * 64,
-                      tq.qb * kTile, tq.h, tq.b);
+                      args.prob[tq.p].q_row0 + tq.qb * kTile, tq.h, tq.b);
         if (qs) ++q_issued1; else ++q_issued0;
       };
-      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
+      for (TileCursor c = first; c.t < total && ok; cursor_next<MULTI>(c, args, total, false)) {
         if (c.n == 0) continue;
-        const TileCoord tc = tile_coord(c.t, args);
+        const TileCoord tc = tile_coord<MULTI>(c.t, args);
         if (has_prologue(c)) {
           load_q(c.k, tc);
           for (int jj = 0; jj < n_prologue(c) && ok; ++jj)
@@ -375,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileCoord tn{};
         if (feeds_next(c)) {
           do {
-            cursor_next(nx, args, total, false);
+            cursor_next<MULTI>(nx, args, total, false);
           } while (nx.t < total && nx.n == 0);
-          tn = tile_coord(nx.t, args);
+          tn = tile_coord<MULTI>(nx.t, args);
         }
         const int nk = own_k(c);
         for (int j = 0; j < c.n && ok; ++j) {
@@ -426,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       int last1 = -1, last2 = -1;  // last two groups of the previous non-empty tile
-      for (TileCursor c = first; c.t < total && ok; cursor_next(c, args, total, false)) {
+      for (TileCursor c = first; c.t < total && ok; cursor_next<MULTI>(c, args, total, false)) {
         if (c.n == 0) continue;
         const int nk = own_k(c);
         if (me == 0 && has_prologue(c)) {
@@ -492,10 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float csc = args.scale_log2;
     bool good = true;
 
-    for (TileCursor c = first; c.t < total; cursor_next(c, args, total, threadIdx.x == 0)) {
+    for (TileCursor c = first; c.t < total; cursor_next<MULTI>(c, args, total, threadIdx.x == 0)) {
+      const Problem& pr = args.prob[MULTI ? c.p : 0];
       float m_own = -INFINITY;  // reference of this group's row sum
       float l_own = 0.f;
-      const int c_qb = TOK ? c.t % args.nqb : 0;
+      const int c_qb = TOK ? (c.t - pr.tile0) % pr.nqb : 0;
       for (int j = ((c.J0 & 1) == g) ? 0 : 1; j < c.n && good; j += 2) {
         const int J = c.J0 + j;
         const int kb = __ldg(c.list + j);
@@ -507,11 +541,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         int valid = kTile;
-        if (kb < 0 || kb >= args.nkb) {
+        if (kb < 0 || kb >= pr.nkb) {
           valid = 0;
           if (row == 0 && dev_status) atomicOr(dev_status, 0x1);
-        } else if ((kb + 1) * kTile > args.Lkv) {
-          valid = args.Lkv - kb * kTile;
+        } else if ((kb + 1) * kTile > pr.Lkv) {
+          valid = pr.Lkv - kb * kTile;
         }
         // with a fine block grid, bit i of `keep` keeps this row's columns
         // [i << mask_shift, (i + 1) << mask_shift) of the tile
@@ -520,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (args.tile_mask) {
           const int fg = kTile >> args.mask_shift;
           const uint32_t full = (1u << fg) - 1u;
-          const uint64_t mk = __ldg(args.tile_mask + (c.list - args.kv_idx) + j);
+          const uint64_t mk = __ldg(args.tile_mask + (c.list - pr.kv_idx) + j);
           keep = static_cast<uint32_t>(mk >> ((row >> args.mask_shift) * fg)) & full;
           fine = __any_sync(0xffffffffu, keep != full);
           keep |= ~full;
@@ -530,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (TOK) {
           const int grow = c_qb * kTile + row;
           const int sk = args.tok.side[args.tok.q_scale];
-          const int gq = grow < args.Lq ? grow : 0;
+          const int gq = grow < pr.Lq ? grow : 0;
           if (valid > 0)
             csla_row_mask(args.tok, gq / sk, gq % sk, kb * kTile, kb * kTile + valid, km);
           fine = true;
@@ -711,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       tc_fence_after();
       const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
-      const TileCoord tc = tile_coord(c.t, args);
+      const TileCoord tc = tile_coord<MULTI>(c.t, args);
       const int grow = tc.qb * kTile + row;
       float l = 0.f, m = -INFINITY, inv_l = 0.f;
       if (c.n > 0) {
@@ -722,8 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = xch[2 * kTile + row] * sa + xch[3 * kTile + row] * sb;
         inv_l = l > 0.f ? 1.f / l : 0.f;
       }
-      if (!aborted && g == 0 && args.lse && grow < args.Lq) {
-        args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.Lq + grow] =
+      if (!aborted && g == 0 && args.lse && grow < pr.Lq) {
+        args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.lse_rows + pr.q_row0 + grow] =
             l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
       if (c.n > 0) {
@@ -758,12 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 0 && !aborted) {
 #pragma unroll
           for (int ch = 0; ch < L::kChunks; ++ch)
-            tma_store_4d(&tm_o, sQ(c.k) + ch * L::kChunkBytes, ch * 64, tc.qb * kTile, tc.h, tc.b);
+            tma_store_4d(&tm_os.m[MULTI ? tc.p : 0], sQ(c.k) + ch * L::kChunkBytes, ch * 64,
+                         tc.qb * kTile, tc.h, tc.b);
           bulk_commit_group();
         }
-      } else if (!aborted && grow < args.Lq) {
+      } else if (!aborted && grow < pr.Lq) {
         // empty list: zero rows (the Q buffer may already hold the next tile's Q)
-        __nv_bfloat16* orow = args.o + tc.b * args.o_sb + tc.h * args.o_sh + grow * args.o_sr;
+        __nv_bfloat16* orow =
+            args.o + tc.b * args.o_sb + tc.h * args.o_sh + (pr.q_row0 + grow) * args.o_sr;
 #pragma unroll
         for (int v = 0; v < D / 16; ++v)
           reinterpret_cast<uint4*>(orow + g * (D / 2))[v] = make_uint4(0u, 0u, 0u, 0u);

@@ -139,10 +139,11 @@ int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   return SPARVAR_OK;
 }
 
-template <int D, bool TOK>
+template <int D, bool TOK, bool MULTI>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const CUtensorMap& to, const sparvar::fwd::Args& a, cudaStream_t stream) {
-  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK>;
+                      const sparvar::fwd::OutMaps& to, const sparvar::fwd::Args& a,
+                      cudaStream_t stream) {
+  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -152,12 +153,14 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
-  const int64_t tiles = static_cast<int64_t>(a.B) * a.H * a.nqb;
+  const int64_t tiles = a.total_tiles;
   const int64_t grid = tiles < sms ? tiles : sms;
   // the kernel's per-CTA sequence counters (blocks, ring positions) are 32-bit
-  if (ceil_div(tiles, grid) * (3 * static_cast<int64_t>(a.idx_row_len) + 1) >= (int64_t{1} << 31))
-    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %d too large per SM",
-                static_cast<long long>(tiles), a.idx_row_len);
+  int64_t row_len = 0;
+  for (int i = 0; i < a.n_problems; ++i) row_len = std::max<int64_t>(row_len, a.prob[i].idx_row_len);
+  if (ceil_div(tiles, grid) * (3 * row_len + 1) >= (int64_t{1} << 31))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %lld too large per SM",
+                static_cast<long long>(tiles), static_cast<long long>(row_len));
   kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
@@ -381,33 +384,40 @@ static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, f
     return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
 
   sparvar::fwd::Args a{};
-  a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
-  a.nqb = static_cast<int>(ceil_div(Lq, 128));
-  a.nkb = static_cast<int>(ceil_div(Lkv, 128));
+  a.B = B; a.H = H; a.n_problems = 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.kv_cnt = kv_cnt; a.kv_idx = kv_idx;
-  a.list_sb = list_strides[0]; a.list_sh = list_strides[1];
-  a.idx_row_len = idx_row_len;
+  sparvar::fwd::Problem& pr = a.prob[0];
+  pr.Lq = Lq; pr.Lkv = Lkv;
+  pr.nqb = static_cast<int>(ceil_div(Lq, 128));
+  pr.nkb = static_cast<int>(ceil_div(Lkv, 128));
+  pr.q_row0 = 0; pr.tile0 = 0;
+  pr.kv_cnt = kv_cnt; pr.kv_idx = kv_idx;
+  pr.list_sb = list_strides[0]; pr.list_sh = list_strides[1];
+  pr.idx_row_len = idx_row_len;
+  a.total_tiles = static_cast<int>(static_cast<int64_t>(B) * H * pr.nqb);
   a.tile_mask = tile_mask;
   a.mask_shift = mask_shift;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
   a.lse = lse;
+  a.lse_rows = Lq;
   a.dev_status = dev_status;
   if (tok) a.tok = *tok;
 
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
+  sparvar::fwd::OutMaps to{};
   if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
   if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
   if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
-  if ((rc = make_tmap(&to, o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o"))) return rc;
+  if ((rc = make_tmap(&to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o")))
+    return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tok) {
-    if (D == 128) return launch_fwd_kernel<128, true>(tq, tk, tv, to, a, st);
-    return launch_fwd_kernel<64, true>(tq, tk, tv, to, a, st);
+    if (D == 128) return launch_fwd_kernel<128, true, false>(tq, tk, tv, to, a, st);
+    return launch_fwd_kernel<64, true, false>(tq, tk, tv, to, a, st);
   }
-  if (D == 128) return launch_fwd_kernel<128, false>(tq, tk, tv, to, a, st);
-  return launch_fwd_kernel<64, false>(tq, tk, tv, to, a, st);
+  if (D == 128) return launch_fwd_kernel<128, false, false>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64, false, false>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
@@ -422,6 +432,85 @@ int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, v
   return attn_fwd_impl(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides, v_strides,
                        o_strides, kv_cnt, kv_idx, list_strides, idx_row_len, tile_mask, mask_block,
                        block_q, block_kv, softmax_scale, dev_status, stream, nullptr);
+}
+
+int sparvar_block_sparse_attn_fwd_multi(
+    const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int q_rows,
+    int kv_rows, int D, const int64_t* q_strides, const int64_t* k_strides,
+    const int64_t* v_strides, const int64_t* o_strides, int n_problems, const int32_t* q_row0,
+    const int32_t* lq, const int32_t* lkv, const int32_t* const* kv_cnt,
+    const int32_t* const* kv_idx, const int64_t* list_strides, const int32_t* idx_row_len,
+    float softmax_scale, int32_t* dev_status, void* stream) {
+  if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (q_rows < 1 || kv_rows < 1 || q_rows > (1 << 30) || kv_rows > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "q_rows=%d kv_rows=%d outside [1, 2^30]", q_rows, kv_rows);
+  if (n_problems < 1 || n_problems > sparvar::fwd::kMaxProblems)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "n_problems=%d outside [1, %d]", n_problems,
+                sparvar::fwd::kMaxProblems);
+  if (!q_row0 || !lq || !lkv || !kv_cnt || !kv_idx || !list_strides || !idx_row_len)
+    return fail(SPARVAR_ERR_INVALID_ARG, "a problem array is NULL");
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f))
+    return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  int rc;
+  if ((rc = check_operand(q, q_strides, B, H, q_rows, D, "q"))) return rc;
+  if ((rc = check_operand(k, k_strides, B, H, kv_rows, D, "k"))) return rc;
+  if ((rc = check_operand(v, v_strides, B, H, kv_rows, D, "v"))) return rc;
+  if ((rc = check_operand(o, o_strides, B, H, q_rows, D, "o"))) return rc;
+  sparvar::fwd::Args a{};
+  a.B = B; a.H = H; a.n_problems = n_problems;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  int64_t tiles = 0;
+  for (int i = 0; i < n_problems; ++i) {
+    if (q_row0[i] < 0 || lq[i] < 1 || static_cast<int64_t>(q_row0[i]) + lq[i] > q_rows)
+      return fail(SPARVAR_ERR_INVALID_ARG, "problem %d: query rows [%d, %d + %d) outside [0, %d)", i,
+                  q_row0[i], q_row0[i], lq[i], q_rows);
+    if (lkv[i] < 1 || lkv[i] > kv_rows)
+      return fail(SPARVAR_ERR_INVALID_ARG, "problem %d: Lkv=%d outside [1, %d]", i, lkv[i], kv_rows);
+    if (!kv_cnt[i] || !kv_idx[i] || list_strides[2 * i] < 0 || list_strides[2 * i + 1] < 0 ||
+        idx_row_len[i] < 0)
+      return fail(SPARVAR_ERR_INVALID_ARG, "problem %d: bad lists", i);
+    sparvar::fwd::Problem& pr = a.prob[i];
+    pr.Lq = lq[i]; pr.Lkv = lkv[i];
+    pr.nqb = static_cast<int>(ceil_div(lq[i], 128));
+    pr.nkb = static_cast<int>(ceil_div(lkv[i], 128));
+    pr.q_row0 = q_row0[i];
+    pr.tile0 = static_cast<int>(tiles);
+    pr.kv_cnt = kv_cnt[i]; pr.kv_idx = kv_idx[i];
+    pr.list_sb = list_strides[2 * i]; pr.list_sh = list_strides[2 * i + 1];
+    pr.idx_row_len = idx_row_len[i];
+    tiles += static_cast<int64_t>(B) * H * pr.nqb;
+    if (tiles > (int64_t{1} << 30))
+      return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
+  }
+  a.total_tiles = static_cast<int>(tiles);
+  a.tile_mask = nullptr;
+  a.mask_shift = 7;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
+  a.lse = lse;
+  a.lse_rows = q_rows;
+  a.dev_status = dev_status;
+
+  CUtensorMap tq, tk, tv;
+  sparvar::fwd::OutMaps to{};
+  if ((rc = make_tmap(&tq, q, D, q_rows, H, B, q_strides[2], q_strides[1], q_strides[0], "q")))
+    return rc;
+  if ((rc = make_tmap(&tk, k, D, kv_rows, H, B, k_strides[2], k_strides[1], k_strides[0], "k")))
+    return rc;
+  if ((rc = make_tmap(&tv, v, D, kv_rows, H, B, v_strides[2], v_strides[1], v_strides[0], "v")))
+    return rc;
+  for (int i = 0; i < n_problems; ++i) {
+    // the problem's own rows only, so the last tile's rows past its end are clipped
+    const void* base = static_cast<const __nv_bfloat16*>(o) + q_row0[i] * o_strides[2];
+    if ((rc = make_tmap(&to.m[i], base, D, lq[i], H, B, o_strides[2], o_strides[1], o_strides[0],
+                        "o")))
+      return rc;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return launch_fwd_kernel<128, false, true>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64, false, true>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_csla_token_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -49,6 +49,9 @@ EXPORTS = {
     "sparvar_csla_token_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i64p, _i64p, _i64p,
                                      _i64p, _i32p, _i, _i, _i, _i, _i, _vp, _vp, _i64p, _i, _f,
                                      _vp, _vp], _i),
+    "sparvar_block_sparse_attn_fwd_multi": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
+                                             _i64p, _i64p, _i64p, _i, _i32p, _i32p, _i32p, _vp,
+                                             _vp, _i64p, _i32p, _f, _vp, _vp], _i),
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
@@ -259,6 +262,42 @@ def sparvar_csla_token_attn_fwd(q, k, v, sides, q_scale, n_sink_scales, radius_p
         len(sides), q_scale, n_sink_scales, radius_prev, radius_own, _ptr(kv_cnt), _ptr(kv_idx),
         _i64([sb, sh]), kv_idx.shape[-1], scale, _ptr(dev_status), _stream(q.device)),
         "sparvar_csla_token_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sparvar_block_sparse_attn_fwd_multi(q, k, v, problems, softmax_scale=None, out=None,
+                                        return_lse=False, dev_status=None):
+    """Several problems in one launch.  q [B,H,q_rows,D], k/v [B,H,kv_rows,D] shared;
+    problems = [(q_row0, lq, lkv, kv_cnt, kv_idx), ...] with 128x128 block lists.
+    Returns O [B,H,q_rows,D] (rows of no problem untouched) and, when asked, the LSE."""
+    B, H, q_rows, D = q.shape
+    kv_rows = k.shape[2]
+    if k.shape != (B, H, kv_rows, D) or v.shape != (B, H, kv_rows, D):
+        raise SparvarError("k/v must be [B, H, kv_rows, D] matching q")
+    qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
+    if out is None:
+        out = torch.zeros_like(q, memory_format=torch.contiguous_format)
+    os_ = _bhrd(out, "out")
+    n = len(problems)
+    lse = torch.full((B, H, q_rows), float("-inf"), dtype=torch.float32, device=q.device) \
+        if return_lse else None
+    r0 = (ctypes.c_int32 * n)(*[p[0] for p in problems])
+    lq = (ctypes.c_int32 * n)(*[p[1] for p in problems])
+    lkv = (ctypes.c_int32 * n)(*[p[2] for p in problems])
+    cnts = (ctypes.c_void_p * n)(*[p[3].data_ptr() for p in problems])
+    idxs = (ctypes.c_void_p * n)(*[p[4].data_ptr() for p in problems])
+    strides, rows = [], []
+    for (_, _, _, cnt, idx) in problems:
+        if cnt.dtype != torch.int32 or idx.dtype != torch.int32 or not idx.is_contiguous():
+            raise SparvarError("kv_cnt/kv_idx must be int32, kv_idx contiguous")
+        strides += list(_list_strides(cnt, B, H))
+        rows.append(idx.shape[-1])
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    _check(lib().sparvar_block_sparse_attn_fwd_multi(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, q_rows, kv_rows, D, qs, ks, vs, os_,
+        n, r0, lq, lkv, ctypes.cast(cnts, ctypes.c_void_p), ctypes.cast(idxs, ctypes.c_void_p),
+        _i64(strides), (ctypes.c_int32 * n)(*rows), scale, _ptr(dev_status), _stream(q.device)),
+        "sparvar_block_sparse_attn_fwd_multi")
     return (out, lse) if return_lse else out
 
 

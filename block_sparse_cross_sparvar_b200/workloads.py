@@ -3,8 +3,9 @@
 * ``cs4a_full_pass``: all 13 scales of one generation step with CS4A: scales
   1-10 dense (the 32x32 scale also yields the row LSE), the decision on the
   32x32 scale (pooled mass >= 0.95), and the mapped lists for 40x40, 48x48 and
-  64x64; ``cs4a_topk_2d_pass`` the same with the Top-K rule (ratio 0.2) and the
-  scale-aware 2-D mapping.
+  64x64; ``cs4a_topk_2d_pass`` the same with the Top-K rule (ratio 0.2), the
+  scale-aware 2-D mapping and the output cache; ``cs4a_fused_pass`` the Top-K /
+  2-D pass with the scales in two multi-problem launches.
 * ``csla_radius_sweep``: the Infinity-8B-like last two scales (B2 H32) with the
   CSLA locality radius of earlier scales at 1, 2 and 4.
 * ``density_sweep``: the last scale with random block lists at fixed densities
@@ -65,6 +66,50 @@ def time_ms(fn, reps, device, warmup=3):
         torch.cuda.synchronize(device)
         out.append(a.elapsed_time(b))
     return float(np.median(out))
+
+
+def cs4a_fused_pass(device, reps=10, seed=0, B=2, H=16, D=128, topk_ratio=0.2, decision_scale=9):
+    """The 13-scale pass in two attention launches: scales 1-10 (dense, with the
+    decision scale's LSE) as one multi-problem launch, then the decision (Top-K),
+    the 2-D mapping and scales 11-13 as a second multi-problem launch."""
+    sides = inputs.INFINITY_SIDES
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    q_all, k_all, v_all = _dev(d["q"], device), _dev(d["k"], device), _dev(d["v"], device)
+    del d
+    n_scales = len(sides)
+    out = torch.zeros_like(q_all)
+    dense = []
+    for s in range(decision_scale + 1):
+        cnt, idx = _dense_lists(-(-(off[s + 1] - off[s]) // 128), -(-off[s + 1] // 128), device)
+        dense.append((off[s], off[s + 1] - off[s], off[s + 1], cnt, idx))
+    state = {}
+
+    def run():
+        _, lse = ops.sparvar_block_sparse_attn_fwd_multi(q_all, k_all, v_all, dense, out=out,
+                                                         return_lse=True)
+        dec = decision_scale
+        dc, di, _ = ops.sparvar_decide_blocks(
+            q_all[:, :, off[dec]:off[dec + 1]], k_all[:, :, :off[dec + 1]], 0.95,
+            lse=lse[:, :, off[dec]:off[dec + 1]].contiguous(), topk_ratio=topk_ratio)
+        late = []
+        for s in range(dec + 1, n_scales):
+            mc, mi, _ = ops.sparvar_map_indices_2d(dc, di, sides, dec, s, 128, 128, off[5])
+            state[s] = (mc, mi)
+            late.append((off[s], off[s + 1] - off[s], off[s + 1], mc, mi))
+        ops.sparvar_block_sparse_attn_fwd_multi(q_all, k_all, v_all, late, out=out)
+
+    ms = time_ms(run, reps, device)
+    flops = 0
+    per_scale = {}
+    for s in range(n_scales):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        f = 4 * nq * L * D * B * H if s <= decision_scale else kept_flops(*state[s], nq, L, 128, D)[0]
+        per_scale[f"{sides[s]}x{sides[s]}"] = {"gflop": f / 1e9, "density": f / (4 * nq * L * D * B * H)}
+        flops += f
+    return {"workload": "cs4a_13_scales_two_launches_2d_mapping", "B": B, "H": H, "D": D,
+            "selection": f"topk {topk_ratio}", "ms": ms, "gflop": flops / 1e9,
+            "tflops": flops / (ms * 1e-3) / 1e12, "scales": per_scale}
 
 
 def cs4a_topk_2d_pass(device, reps=10, seed=0):

@@ -264,6 +264,32 @@ SPARVAR_API int sparvar_coarsen_lists(const int32_t* kv_cnt, const int32_t* kv_i
                                       int32_t* dev_status, void* stream);
 
 /*
+ * Several block-sparse attention problems in one launch (for instance the scales
+ * of one generation step, which share the Q, K and V tensors of the whole
+ * multi-scale sequence): the persistent kernel walks the query tiles of all
+ * problems as one work list, so small scales do not each pay a launch and a
+ * tail.  Problem i is sparvar_block_sparse_attn_fwd on query rows
+ * [q_row0[i], q_row0[i] + lq[i]) of q and o, keys [0, lkv[i]) of k and v, with
+ * lists kv_cnt[i], kv_idx[i] (device pointers in host arrays), list strides
+ * list_strides[2i], list_strides[2i+1] and row length idx_row_len[i]; the blocks
+ * are 128 x 128 (no fine grids).
+ *
+ * q, o [B][H][q_rows][D]; k, v [B][H][kv_rows][D]: device bf16, strides and
+ * alignment as for sparvar_block_sparse_attn_fwd, D in {64, 128}.  lse device
+ * fp32 [B][H][q_rows] or NULL (rows of no problem are not written).  1 <=
+ * n_problems <= 16; query row ranges must not overlap.  The problems' results
+ * are those of separate calls (up to the order in which PV products reach the
+ * accumulator).
+ */
+SPARVAR_API int sparvar_block_sparse_attn_fwd_multi(
+    const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int q_rows,
+    int kv_rows, int D, const int64_t* q_strides, const int64_t* k_strides,
+    const int64_t* v_strides, const int64_t* o_strides, int n_problems, const int32_t* q_row0,
+    const int32_t* lq, const int32_t* lkv, const int32_t* const* kv_cnt,
+    const int32_t* const* kv_idx, const int64_t* list_strides, const int32_t* idx_row_len,
+    float softmax_scale, int32_t* dev_status, void* stream);
+
+/*
  * Block-sparse attention with the CSLA token mask applied inside the kept tiles
  * ("Methodology in Plain English", CSLA paragraph: the token-wise mask, here used
  * as it is rather than only through its blocks): O[q] = sum_key softmax(s(q,key)) V[key] over the keys the CSLA token

@@ -615,3 +615,51 @@ def test_csla_token_attention_last_scale_sampled_rows():
     rng = np.random.default_rng(5)
     rows = np.unique(np.concatenate([rng.integers(0, 4096, 48), [0, 63, 64, 4095]]))
     _token_check(INF, 12, 5, 2, 4, 2, 2, 128, 7, rows=rows)
+
+
+# ------------------------------------------------------------------ several problems per launch
+def _dense_lists(nq, L):
+    nqb, nkb = -(-nq // 128), -(-L // 128)
+    cnt = torch.full((nqb,), nkb, dtype=torch.int32, device="cuda")
+    idx = torch.arange(nkb, dtype=torch.int32, device="cuda").repeat(nqb, 1).contiguous()
+    return cnt, idx, np.ones((nqb, nkb), bool)
+
+
+@pytest.mark.parametrize("sides,first_sparse,D,B,H", [(INF, 10, 128, 1, 2), (TINY, 3, 64, 1, 2)])
+def test_multi_problem_launch(sides, first_sparse, D, B, H):
+    """Every scale of a schedule in one launch over the shared multi-scale Q/K/V:
+    dense for the early scales, CSLA lists for the late ones; each scale's rows,
+    including the ragged last tile next to the following scale, against the oracle."""
+    ns = 5 if sides is INF else 2
+    rp, ro = (2, 4) if sides is INF else (1, 1)
+    d = inputs.make_qkv(40 + D, B, H, sides, D, ns, pe=sides is INF)
+    off = d["offsets"]
+    q, k, v = _dev(d["q"]), _dev(d["k"]), _dev(d["v"])
+    problems, blks = [], []
+    for s in range(len(sides)):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        if s < first_sparse:
+            cnt, idx, blk = _dense_lists(nq, L)
+        else:
+            cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, ns, rp, ro, 128, 128)
+            _, _, blk = orc.build_csla_mask(sides, s, ns, rp, ro, 128, 128)
+        problems.append((off[s], nq, L, cnt, idx))
+        blks.append(blk)
+    st = _status()
+    o, lse = ops.sparvar_block_sparse_attn_fwd_multi(q, k, v, problems, return_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    rng = np.random.default_rng(D)
+    for s in range(len(sides)):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        rows = np.arange(nq) if nq <= 600 else np.unique(np.concatenate(
+            [rng.integers(0, nq, 40), [0, nq - 1, (nq - 1) // 128 * 128]]))
+        for b in range(B):
+            for h in range(H):
+                O, Lo = orc.masked_attention_rows(rows, q_bits_f(d["q"][:, :, off[s]:off[s + 1]], b, h),
+                                                  q_bits_f(d["k"][:, :, :L], b, h),
+                                                  q_bits_f(d["v"][:, :, :L], b, h), blks[s], 128, 128)
+                err = np.abs(o[b, h, off[s] + rows] - O)
+                assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (s, b, h, err.max())
+                assert np.abs(lse[b, h, off[s] + rows] - Lo).max() < 1e-3

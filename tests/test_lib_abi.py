@@ -156,3 +156,23 @@ def test_ocache_rejects_bad_arguments(lib):
     assert call(s_src=0) == 1
     assert call(ot=0) == 1 and "o_target" in lib.sparvar_last_error().decode()
     assert call(od=8) == 1 and "aligned" in lib.sparvar_last_error().decode()
+
+
+def test_multi_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    i64 = lambda *x: (ctypes.c_int64 * len(x))(*x)  # noqa: E731
+    i32 = lambda *x: (ctypes.c_int32 * len(x))(*x)  # noqa: E731
+    st = i64(0, 0, 128)
+    ptrs = (ctypes.c_void_p * 2)(16, 16)
+
+    def call(n=2, r0=(0, 100), lq=(100, 200), lkv=(300, 500), q_rows=300, D=128):
+        return lib.sparvar_block_sparse_attn_fwd_multi(
+            vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, q_rows, 500, D, st, st, st, st, n, i32(*r0),
+            i32(*lq), i32(*lkv), ctypes.cast(ptrs, vp), ctypes.cast(ptrs, vp), i64(0, 0, 0, 0),
+            i32(4, 4), 0.1, vp(0), vp(0))
+
+    assert call(n=17) == 2 and "n_problems" in lib.sparvar_last_error().decode()
+    assert call(n=0) == 2
+    assert call(r0=(0, 250)) == 1 and "problem 1" in lib.sparvar_last_error().decode()
+    assert call(lkv=(300, 501)) == 1 and "Lkv=501" in lib.sparvar_last_error().decode()
+    assert call(D=96) == 2
