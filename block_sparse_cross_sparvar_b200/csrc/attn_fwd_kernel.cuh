@@ -158,6 +158,7 @@ struct TileCursor {
 
 struct TileCoord {
   int p, b, h, qb;
+  int nkb, row0;  // the problem's key-block count and first query row
 };
 template <bool MULTI>
 __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
@@ -165,10 +166,10 @@ __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
   if constexpr (MULTI) {
     while (p + 1 < a.n_problems && t >= a.prob[p + 1].tile0) ++p;
   }
-  const Problem& pr = a.prob[p];
-  const int lt = t - pr.tile0;
-  const int bh = lt / pr.nqb;
-  return TileCoord{p, bh / a.H, bh % a.H, lt % pr.nqb};
+  const int nqb = a.prob[p].nqb;
+  const int lt = MULTI ? t - a.prob[p].tile0 : t;  // a single problem starts at tile 0, row 0
+  const int bh = lt / nqb;
+  return TileCoord{p, bh / a.H, bh % a.H, lt % nqb, a.prob[p].nkb, MULTI ? a.prob[p].q_row0 : 0};
 }
 
 template <bool MULTI>
@@ -371,8 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return;
         }
         relg_sh[s] = grp;
-        const int nkb_p = args.prob[tc.p].nkb;
-        kb = kb < 0 ? -1 : (kb > nkb_p ? nkb_p : kb);
+        kb = kb < 0 ? -1 : (kb > tc.nkb ? tc.nkb : kb);
         mbar_arrive_expect_tx(&bars.full[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < L::kChunks; ++cc)
           tma_load_4d(sQ(k) + cc * L::kChunkBytes, &tm_q, &bars.q_full[qs], cc * 64,
-                      args.prob[tq.p].q_row0 + tq.qb * kTile, tq.h, tq.b);
+                      tq.row0 + tq.qb * kTile, tq.h, tq.b);
         if (qs) ++q_issued1; else ++q_issued0;
       };
       for (TileCursor c = first; c.t < total && ok; cursor_next<MULTI>(c, args, total, false)) {
@@ -526,10 +526,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool good = true;
 
     for (TileCursor c = first; c.t < total; cursor_next<MULTI>(c, args, total, threadIdx.x == 0)) {
-      const Problem& pr = args.prob[MULTI ? c.p : 0];
+      // the tile's problem, read once per tile into registers
+      const int pi = MULTI ? c.p : 0;
+      const int p_nkb = args.prob[pi].nkb, p_lkv = args.prob[pi].Lkv, p_lq = args.prob[pi].Lq;
+      const int p_row0 = MULTI ? args.prob[pi].q_row0 : 0;
       float m_own = -INFINITY;  // reference of this group's row sum
       float l_own = 0.f;
-      const int c_qb = TOK ? (c.t - pr.tile0) % pr.nqb : 0;
+      const int c_qb = TOK ? (c.t - args.prob[pi].tile0) % args.prob[pi].nqb : 0;
       for (int j = ((c.J0 & 1) == g) ? 0 : 1; j < c.n && good; j += 2) {
         const int J = c.J0 + j;
         const int kb = __ldg(c.list + j);
@@ -541,11 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         int valid = kTile;
-        if (kb < 0 || kb >= pr.nkb) {
+        if (kb < 0 || kb >= p_nkb) {
           valid = 0;
           if (row == 0 && dev_status) atomicOr(dev_status, 0x1);
-        } else if ((kb + 1) * kTile > pr.Lkv) {
-          valid = pr.Lkv - kb * kTile;
+        } else if ((kb + 1) * kTile > p_lkv) {
+          valid = p_lkv - kb * kTile;
         }
         // with a fine block grid, bit i of `keep` keeps this row's columns
         // [i << mask_shift, (i + 1) << mask_shift) of the tile
@@ -554,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (args.tile_mask) {
           const int fg = kTile >> args.mask_shift;
           const uint32_t full = (1u << fg) - 1u;
-          const uint64_t mk = __ldg(args.tile_mask + (c.list - pr.kv_idx) + j);
+          const uint64_t mk = __ldg(args.tile_mask + (c.list - args.prob[pi].kv_idx) + j);
           keep = static_cast<uint32_t>(mk >> ((row >> args.mask_shift) * fg)) & full;
           fine = __any_sync(0xffffffffu, keep != full);
           keep |= ~full;
@@ -564,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (TOK) {
           const int grow = c_qb * kTile + row;
           const int sk = args.tok.side[args.tok.q_scale];
-          const int gq = grow < pr.Lq ? grow : 0;
+          const int gq = grow < p_lq ? grow : 0;
           if (valid > 0)
             csla_row_mask(args.tok, gq / sk, gq % sk, kb * kTile, kb * kTile + valid, km);
           fine = true;
@@ -756,8 +759,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = xch[2 * kTile + row] * sa + xch[3 * kTile + row] * sb;
         inv_l = l > 0.f ? 1.f / l : 0.f;
       }
-      if (!aborted && g == 0 && args.lse && grow < pr.Lq) {
-        args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.lse_rows + pr.q_row0 + grow] =
+      if (!aborted && g == 0 && args.lse && grow < p_lq) {
+        args.lse[(static_cast<int64_t>(tc.b) * args.H + tc.h) * args.lse_rows + p_row0 + grow] =
             l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
       if (c.n > 0) {
@@ -796,10 +799,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                          tc.qb * kTile, tc.h, tc.b);
           bulk_commit_group();
         }
-      } else if (!aborted && grow < pr.Lq) {
+      } else if (!aborted && grow < p_lq) {
         // empty list: zero rows (the Q buffer may already hold the next tile's Q)
         __nv_bfloat16* orow =
-            args.o + tc.b * args.o_sb + tc.h * args.o_sh + (pr.q_row0 + grow) * args.o_sr;
+            args.o + tc.b * args.o_sb + tc.h * args.o_sh + (p_row0 + grow) * args.o_sr;
 #pragma unroll
         for (int v = 0; v < D / 16; ++v)
           reinterpret_cast<uint4*>(orow + g * (D / 2))[v] = make_uint4(0u, 0u, 0u, 0u);
