@@ -242,6 +242,31 @@ def test_attention_dense_lists_and_random_lists_per_head():
     _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D, scale=0.11)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_persistent_short_and_empty_lists(D):
+    """Many query tiles per CTA (2 x 16 x 40 = 1280 tiles on at most one CTA per SM)
+    with lists of 0-6 blocks in random order, so that each CTA walks every kind of
+    transition: empty tiles between others, tiles of one or two blocks (whose
+    first score MMAs are issued on their own) and tiles of three or more (which
+    feed the next one); ragged query and key tails; every row of every head."""
+    rng = np.random.default_rng(17 + D)
+    B, H = 2, 16
+    nqb, nkb = 40, 6
+    Lq, Lkv = nqb * 128 - 37, nkb * 128 - 50
+    bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
+            for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
+    lens = rng.choice(nkb + 1, size=(B, H, nqb), p=[0.15, 0.2, 0.2, 0.15, 0.1, 0.1, 0.1])
+    lens[0, 0, :4] = [0, 0, 3, 0]  # a feeding tile whose successors are empty
+    idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                idx_np[b, h, qb, :lens[b, h, qb]] = rng.permutation(nkb)[:lens[b, h, qb]]
+    cnt = torch.from_numpy(lens.astype(np.int32)).cuda()
+    idx = torch.from_numpy(idx_np).cuda()
+    _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D)
+
+
 def test_attention_unordered_lists_give_same_result():
     d = inputs.make_qkv(3, 1, 2, INF, 128, 5)
     off = d["offsets"]
