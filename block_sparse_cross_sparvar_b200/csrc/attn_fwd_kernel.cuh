@@ -316,7 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
   volatile int* abort_flag = &abort_sh;
   int32_t* dev_status = args.dev_status;
-  const int total = args.total_tiles;
+  // a single problem's tile count is its shape's (equal to total_tiles); written so,
+  // the compiler relates tile ids to tile coordinates and emits shorter tile code
+  const int total = MULTI ? args.total_tiles : args.B * args.H * args.prob[0].nqb;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
