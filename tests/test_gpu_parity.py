@@ -5,7 +5,6 @@ margin rule: rows whose decision sits within 1e-4 of a flip are checked for
 validity instead).  Attention outputs must match with max-abs <= 2e-2 and
 mean-abs <= 2e-3 against fp64 on the same bf16 inputs.
 """
-import math
 
 import numpy as np
 import pytest

@@ -5,7 +5,6 @@ restatement of the mapping on token level, and invariants that the method's
 description fixes (sinks always kept, own token always kept, radius >= side is
 dense, mapping identity, ranges, monotonicity).
 """
-import itertools
 import math
 import os
 from fractions import Fraction
