@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsparvar.so")
 SOURCES = ["sparvar_api.cu"]
 HEADERS = ["attn_fwd_kernel.cuh", "attn_kernel.cuh", "mask_kernels.cuh", "ocache_kernel.cuh", "ptx.cuh",
-           "tmem_io.cuh"]
+           "tmem_io.cuh", "wait_probe_kernel.cuh"]
 
 
 def nvcc_path() -> str:

@@ -17,6 +17,7 @@
 #include "attn_kernel.cuh"
 #include "mask_kernels.cuh"
 #include "ocache_kernel.cuh"
+#include "wait_probe_kernel.cuh"
 
 // Scratch of sparvar_block_sparse_attn_fwd_static: one array per device, in the
 // library's own module, shared by every call on that device.
@@ -342,6 +343,19 @@ int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_r
       kv_cnt, kv_idx, n_rows, idx_row_len, nkb, dev_status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "validate_lists_kernel launch");
+  return SPARVAR_OK;
+}
+
+int sparvar_wait_timeout_probe(uint64_t limit_ns, int32_t* dev_status, int32_t* result,
+                               void* stream) {
+  if (!dev_status || !result) return fail(SPARVAR_ERR_INVALID_ARG, "dev_status/result is NULL");
+  if (limit_ns < 1000u || limit_ns > 1000000000u)
+    return fail(SPARVAR_ERR_INVALID_ARG, "limit_ns=%llu outside [1e3, 1e9]",
+                static_cast<unsigned long long>(limit_ns));
+  sparvar::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      limit_ns, SPARVAR_DEV_TIMEOUT, dev_status, result);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait_probe_kernel launch");
   return SPARVAR_OK;
 }
 

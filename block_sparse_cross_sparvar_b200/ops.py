@@ -55,6 +55,7 @@ EXPORTS = {
     "sparvar_coarsen_lists": ([_vp, _vp, _i64p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp],
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
+    "sparvar_wait_timeout_probe": ([ctypes.c_uint64, _vp, _vp, _vp], _i),
 }
 
 
@@ -387,6 +388,20 @@ def sparvar_map_indices_2d(src_cnt, src_idx, sides, src_scale, dst_scale, block_
         block_kv, n_sink_tokens, _ptr(cnt), _ptr(idx), _ptr(mask), _ptr(dev_status), _stream(dev)),
         "sparvar_map_indices_2d")
     return cnt, idx, mask
+
+
+def sparvar_wait_timeout_probe(limit_ns, device="cuda"):
+    """Run the bounded-wait self-test on `device`: a wait that nothing completes
+    gives up after `limit_ns`.  Returns (status bits, completed, abort flag,
+    microseconds waited) (synchronises)."""
+    device = torch.device(device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    result = torch.full((3,), -1, dtype=torch.int32, device=device)
+    _check(lib().sparvar_wait_timeout_probe(int(limit_ns), _ptr(status), _ptr(result),
+                                            _stream(device)),
+           "sparvar_wait_timeout_probe")
+    r = result.cpu().tolist()
+    return int(status.item()), r[0], r[1], r[2]
 
 
 def sparvar_validate_lists(kv_cnt, kv_idx, nkb):

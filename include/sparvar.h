@@ -376,6 +376,22 @@ SPARVAR_API int sparvar_block_sparse_attn_fwd_static(
 SPARVAR_API int sparvar_validate_lists(const int32_t* kv_cnt, const int32_t* kv_idx, int n_rows,
                            int idx_row_len, int nkb, int32_t* dev_status, void* stream);
 
+/*
+ * Self-test of the failure path every kernel of the library shares (no
+ * counterpart in the pages): one GPU thread waits on a shared-memory mbarrier
+ * that nothing completes, using the same bounded wait as the attention
+ * pipeline.  After limit_ns nanoseconds (1e3 <= limit_ns <= 1e9) it gives up,
+ * ORs SPARVAR_DEV_TIMEOUT into *dev_status and returns; the CUDA context stays
+ * usable.  result (device int32[3], written): [0] 1 if the wait completed
+ * (never expected), 0 if it gave up; [1] the CTA's abort flag afterwards (1);
+ * [2] microseconds spent waiting.  dev_status and result are device pointers
+ * owned by the caller; nothing is synchronised.  Returns SPARVAR_ERR_INVALID_ARG
+ * for null pointers or a limit outside the range, SPARVAR_ERR_CUDA on a launch
+ * failure.
+ */
+SPARVAR_API int sparvar_wait_timeout_probe(uint64_t limit_ns, int32_t* dev_status,
+                                           int32_t* result, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -687,3 +687,21 @@ def test_multi_problem_launch(sides, first_sparse, D, B, H):
                 err = np.abs(o[b, h, off[s] + rows] - O)
                 assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (s, b, h, err.max())
                 assert np.abs(lse[b, h, off[s] + rows] - Lo).max() < 1e-3
+
+
+# ------------------------------------------------------------------ failure path
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """A wait that nothing completes gives up after its limit, raises the abort
+    flag and reports SPARVAR_DEV_TIMEOUT; attention launched right after on the
+    same context is still correct."""
+    limit_ns = 2_000_000
+    status, completed, abort, waited_us = ops.sparvar_wait_timeout_probe(limit_ns)
+    assert status == 0x2 and completed == 0 and abort == 1
+    assert limit_ns // 1000 <= waited_us < 1_000_000
+    rng = np.random.default_rng(23)
+    B, H, Lq, Lkv, D = 1, 2, 200, 300, 128
+    bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
+            for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
+    cnt = torch.tensor([3, 2], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[0, 1, 2], [2, 0, -1]], dtype=torch.int32, device="cuda")
+    _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D)

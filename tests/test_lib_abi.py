@@ -176,3 +176,12 @@ def test_multi_rejects_bad_arguments(lib):
     assert call(r0=(0, 250)) == 1 and "problem 1" in lib.sparvar_last_error().decode()
     assert call(lkv=(300, 501)) == 1 and "Lkv=501" in lib.sparvar_last_error().decode()
     assert call(D=96) == 2
+
+
+def test_wait_probe_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    assert lib.sparvar_wait_timeout_probe(10**6, vp(0), vp(16), vp(0)) == 1
+    assert lib.sparvar_wait_timeout_probe(10**6, vp(16), vp(0), vp(0)) == 1
+    assert lib.sparvar_wait_timeout_probe(999, vp(16), vp(16), vp(0)) == 1
+    assert "limit_ns=999" in lib.sparvar_last_error().decode()
+    assert lib.sparvar_wait_timeout_probe(10**9 + 1, vp(16), vp(16), vp(0)) == 1
