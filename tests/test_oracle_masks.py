@@ -387,3 +387,20 @@ def test_map_2d_identity_and_invariants():
     assert np.all(orc.map_block_mask_2d(more, sides, 9, 12, 128, 128, 121) >= dst)
     cnt, idx, blk = orc.map_indices_2d(*orc.block_lists(src), sides, 9, 12, 128, 128, 121)
     assert np.array_equal(blk, dst)
+
+
+def test_block_lists_layout_and_inverse():
+    """Lists are ascending with a -1 tail and counts equal to the kept blocks per
+    row (a hand-made mask); lists_to_blocks inverts them and ignores entry order
+    and the tail."""
+    blk = np.array([[1, 0, 1, 1], [0, 0, 0, 0], [0, 1, 0, 0]], dtype=bool)
+    cnt, idx = orc.block_lists(blk)
+    assert cnt.tolist() == [3, 0, 1]
+    assert idx.tolist() == [[0, 2, 3, -1], [-1, -1, -1, -1], [1, -1, -1, -1]]
+    assert np.array_equal(orc.lists_to_blocks(cnt, idx, 4), blk)
+    shuffled = np.array([[3, 0, 2, -1], [-1, -1, -1, -1], [1, -1, -1, -1]], dtype=np.int32)
+    assert np.array_equal(orc.lists_to_blocks(cnt, shuffled, 4), blk)
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        r = rng.random((5, 9)) < rng.random()
+        assert np.array_equal(orc.lists_to_blocks(*orc.block_lists(r), 9), r)
