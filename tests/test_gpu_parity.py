@@ -255,7 +255,13 @@ def test_attention_persistent_short_and_empty_lists(D):
     bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
             for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
     lens = rng.choice(nkb + 1, size=(B, H, nqb), p=[0.15, 0.2, 0.2, 0.15, 0.1, 0.1, 0.1])
-    lens[0, 0, :4] = [0, 0, 3, 0]  # a feeding tile whose successors are empty
+    # CTA 1 walks tiles 1, 1 + G, 1 + 2G, ... (G = one CTA per SM): a tile that
+    # feeds the next, two empty tiles, a two-block tile, a feeding tile again
+    G = torch.cuda.get_device_properties(0).multi_processor_count
+    flat = lens.reshape(-1)
+    for i, n in enumerate([3, 0, 0, 2, 4]):
+        if 1 + i * G < flat.size:
+            flat[1 + i * G] = n
     idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
     for b in range(B):
         for h in range(H):
