@@ -325,7 +325,7 @@ def main():
                        "kept_gflop_per_step_per_gpu": flops_step / 1e9,
                        "l2": "256 MB flush write between timed steps",
                        "parallelism": f"independent batch per GPU x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128, TOK=false, MULTI=false>",
                          "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16"],
                          "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']}",
