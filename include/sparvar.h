@@ -118,7 +118,7 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
  * kept (every block when the total stays below it).  With topk_ratio > 0 the
  * first k = ceil(topk_ratio * nkb) blocks of that order are kept instead (at
  * least one; the product is taken with a 1e-6 allowance so 0.2 * 20 gives 4):
- * the Top-K rule of the same paragraph, "Top-K around 0.2" in "Main Findings".
+ * the Top-K rule of the same paragraph, with the ratio 0.2 of "Main Findings".
  * Kept lists are written in ascending order.
  *
  * q [B][H][Lq][D], k [B][H][Lkv][D]: device bf16; strides in elements for
@@ -315,9 +315,10 @@ SPARVAR_API int sparvar_csla_token_attn_fwd(const void* q, const void* k, const 
                                             void* stream);
 
 /*
- * CS4A output cache ("Methodology in Plain English", CS4A paragraph: the residual
- * output left at the decision scale is cached and upsampled to correct the
- * later sparse outputs; "Main Findings": O_cache adds about 0.7 PSNR):
+ * CS4A output cache ("Methodology in Plain English", CS4A paragraph: what the
+ * sparse computation misses at the decision scale is kept and, brought to a
+ * later scale's grid, corrects that scale's sparse output; "Main Findings":
+ * the cache is worth about 0.7 dB of PSNR):
  *
  *   out[t] = o_target[t] + o_dense[src(t)] - o_sparse[src(t)],
  *

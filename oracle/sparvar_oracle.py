@@ -25,7 +25,7 @@ Conventions (the plainest reading where the pages are silent):
     globally over the key prefix;
   * the softmax scale defaults to 1/sqrt(D);
   * inside a kept block attention is dense; the token mask only decides which
-    blocks are kept ([M] CSLA: the token mask "is then aggregated into blocks").
+    blocks are kept ([M] CSLA: the token rule is reduced to a block rule).
 
 Parity status: every function here is pinned by tests under ``tests/``
 (closed forms, brute force, hand-derived golden fixtures, invariants).
@@ -58,10 +58,10 @@ def n_blocks(n, block):
 def csla_token_mask(sides, q_scale, n_sink_scales, radius_prev, radius_own):
     """Token-wise CSLA mask T[q, key] for the queries of scale ``q_scale``.
 
-    [M] CSLA: "each query at a high-resolution scale is projected onto the
-    coordinate grid of each earlier scale, and attention is allowed only within
-    a per-scale window radius around that projected position.  A separate sink
-    mask keeps a small set of early tokens visible to everything."
+    [M] CSLA: a query of a large scale is mapped to its position on the grid of
+    every earlier scale and may attend there only to keys near that position,
+    within a radius chosen per scale; besides, a few early tokens (the sink)
+    stay visible to every query.
 
     * sink: keys of the first ``n_sink_scales`` scales ([F]: scale <= 5);
     * every later scale m <= q_scale: query (i, j) of the side-s_k grid projects
@@ -287,8 +287,8 @@ def select_blocks_by_mass(M, mass_threshold):
 def topk_count(ratio, nkb):
     """Blocks kept per query block in the Top-K mode.
 
-    [M] CS4A uses "a Top-K operation to find which keys matter most", with
-    "Top-K around 0.2" as the pages' default; read as a ratio of the key blocks:
+    [M] CS4A keeps the most important key blocks by a Top-K choice, and [F]
+    gives 0.2 as its usual ratio; read as a ratio of the key blocks:
     k = ceil(ratio * NKB), at least 1 and at most NKB.  The product is taken with
     a 1e-6 allowance so that a ratio given in binary floating point (0.2 is
     0.2000000030 as a float32) does not round 0.2 * 20 up to 5.
@@ -337,9 +337,9 @@ def decide_blocks(q, k, block_q, block_kv, mass_threshold, scale=None, topk_rati
 def map_block_mask(src_blk, src_nq, src_lkv, dst_nq, dst_lkv, block_q, block_kv, n_sink_tokens):
     """Map kept decision-scale blocks onto a later scale's block grid.
 
-    [M] CS4A: the selected indices "are then mapped to later, larger scales by
-    rescaling the index positions (with an optional concatenation of the sink
-    region)".  Reading: each kept (qb, kb) covers the query-token interval
+    [M] CS4A: the kept block positions found at the decision scale are carried
+    to each later, larger scale by scaling their coordinates, and the sink
+    region may be appended.  Reading: each kept (qb, kb) covers the query-token interval
     [qlo, qhi) and key-token interval [klo, khi); both are rescaled
     proportionally, [floor(lo * N_dst / N_src), ceil(hi * N_dst / N_src)),
     with N the query count for the query axis and the key-prefix length for the
@@ -392,8 +392,9 @@ def map_block_mask_2d(src_blk, sides, src_scale, dst_scale, block_q, block_kv, n
     """Scale-aware 2-D reading of the CS4A mapping (the alternative to
     ``map_block_mask``).
 
-    [M] CS4A maps the selected indices "to later, larger scales by rescaling the
-    index positions" and calls the result scale self-similar.  Reading: a query
+    [M] CS4A carries the kept positions to later, larger scales by scaling their
+    coordinates, relying on the attention pattern looking alike from scale to
+    scale.  Reading: a query
     token (i, j) of the decision scale (side s_d) stands for its upscaled cell of
     the target scale (side s_t): rows upscale_cell(i), columns upscale_cell(j).  A
     key keeps its position when it lies in a scale before the decision scale (the
@@ -469,8 +470,8 @@ def nearest_source(i, s_src, s_dst):
 
 
 def ocache_residual(o_dense, o_sparse):
-    """[M] CS4A keeps "the residual output left over at the decision scale" as a
-    cache.  Reading: the part of the decision scale's dense attention output that
+    """[M] CS4A caches what the sparse computation leaves out at the decision
+    scale.  Reading: the part of the decision scale's dense attention output that
     its own block-sparse output (with the blocks the decision keeps) misses,
     R = O_dense - O_sparse, per token and channel."""
     return np.asarray(o_dense, dtype=np.float64) - np.asarray(o_sparse, dtype=np.float64)
@@ -490,8 +491,8 @@ def ocache_upsample(r, s_src, s_dst):
 
 
 def ocache_apply(o_target, o_dense, o_sparse, s_src, s_dst):
-    """[M] the cache "upsampled to correct the later sparse outputs": a later
-    scale's block-sparse output plus the upsampled decision-scale residual."""
+    """[M] the cached residual, brought up to a later scale's grid, is added to
+    that scale's block-sparse output."""
     return np.asarray(o_target, dtype=np.float64) + ocache_upsample(
         ocache_residual(o_dense, o_sparse), s_src, s_dst)
 
