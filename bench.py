@@ -249,8 +249,9 @@ def main():
         step(q, kk, vv, o)
     torch.cuda.synchronize()
 
-    clocks_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/sparvar_clocks_{rank}.csv"
+    # raw nvidia-smi samples; the JSON line carries their summary
+    clocks_dir = os.environ.get("SPARVAR_CLOCKS_DIR", "/tmp")
+    clocks_path = os.path.join(clocks_dir, f"sparvar_clocks_rank{rank}.csv")
     sampler, sf = start_clock_sampler(clocks_path) if rank == 0 else (None, None)
     t_soak = time.perf_counter()
     while time.perf_counter() - t_soak < args.soak_s:  # same load as the timed steps, untimed
