@@ -695,6 +695,44 @@ def test_multi_problem_launch(sides, first_sparse, D, B, H):
                 assert np.abs(lse[b, h, off[s] + rows] - Lo).max() < 1e-3
 
 
+def test_multi_problem_launch_full_size_sampled():
+    """The 13 Infinity scales at B2 H16 D128 in one launch (2784 query tiles, about
+    19 per CTA, so CTAs cross from one problem to the next mid-sequence): dense
+    lists for scales 1-10, CSLA lists for the last three; sampled rows of every
+    scale for three (batch, head) pairs, and the LSE."""
+    B, H, D = 2, 16, 128
+    d = inputs.make_qkv(7, B, H, INF, D, 5)
+    off = d["offsets"]
+    q, k, v = _dev(d["q"]), _dev(d["k"]), _dev(d["v"])
+    problems, blks = [], []
+    for s in range(len(INF)):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        if s < 10:
+            cnt, idx, blk = _dense_lists(nq, L)
+        else:
+            cnt, idx, _ = ops.sparvar_build_csla_mask(INF, s, 5, 2, 4, 128, 128)
+            _, _, blk = orc.build_csla_mask(INF, s, 5, 2, 4, 128, 128)
+        problems.append((off[s], nq, L, cnt, idx))
+        blks.append(blk)
+    st = _status()
+    o, lse = ops.sparvar_block_sparse_attn_fwd_multi(q, k, v, problems, return_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rng = np.random.default_rng(77)
+    for s in range(len(INF)):
+        nq, L = off[s + 1] - off[s], off[s + 1]
+        rows = np.arange(nq) if nq <= 64 else np.unique(np.concatenate(
+            [rng.integers(0, nq, 12), [0, nq - 1, (nq - 1) // 128 * 128]]))
+        sel = torch.from_numpy(off[s] + rows).cuda()
+        for b, h in [(0, 0), (1, 9), (0, 15)]:
+            O, Lo = orc.masked_attention_rows(rows, q_bits_f(d["q"][:, :, off[s]:off[s + 1]], b, h),
+                                              q_bits_f(d["k"][:, :, :L], b, h),
+                                              q_bits_f(d["v"][:, :, :L], b, h), blks[s], 128, 128)
+            err = np.abs(o[b, h, sel].float().cpu().numpy() - O)
+            assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (s, b, h, err.max())
+            assert np.abs(lse[b, h, sel].cpu().numpy() - Lo).max() < 1e-3
+
+
 # ------------------------------------------------------------------ failure path
 def test_bounded_wait_gives_up_and_the_context_stays_usable():
     """A wait that nothing completes gives up after its limit, raises the abort
