@@ -348,7 +348,8 @@ def main():
             del q, kk, vv, o, hq, hk, hv
             torch.cuda.empty_cache()
             for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass, workloads.cs4a_fused_pass,
-                       workloads.csla_radius_sweep, workloads.density_sweep):
+                       workloads.csla_radius_sweep, workloads.csla_granularity_sweep,
+                       workloads.density_sweep):
                 print(json.dumps({"extra": fn(dev)}), flush=True)
                 torch.cuda.empty_cache()
     if world > 1:

@@ -8,6 +8,8 @@
   2-D pass with the scales in two multi-problem launches.
 * ``csla_radius_sweep``: the Infinity-8B-like last two scales (B2 H32) with the
   CSLA locality radius of earlier scales at 1, 2 and 4.
+* ``csla_granularity_sweep``: the last scale under CSLA with 128x128 blocks,
+  64x64 blocks and the token mask inside 128x128 tiles.
 * ``density_sweep``: the last scale with random block lists at fixed densities
   (sink block always kept), with the full key prefix and with the 40x40 and
   48x48 scales skipped from the prefix.
@@ -204,6 +206,44 @@ def csla_radius_sweep(device, reps=10, seed=0, B=2, H=32, D=128, radii=(1, 2, 4)
                         "tflops": f / (ms * 1e-3) / 1e12})
     return {"workload": "infinity8b_last_two_scales_csla_radius_sweep", "B": B, "H": H, "D": D,
             "runs": res}
+
+
+def csla_granularity_sweep(device, reps=10, seed=0, B=2, H=16, D=128):
+    """The Infinity-2B last scale under CSLA at three granularities: 128x128
+    blocks, 64x64 blocks (coarsened to 128x128 tiles with masks inside the call,
+    the coarsening timed with it), and the token mask applied inside the 128x128
+    tiles.  ``tflops`` counts the kept blocks' work at the run's own block size;
+    for the token mask it counts the executed tiles' work (fewer token pairs are
+    kept than the tiles hold)."""
+    sides = inputs.INFINITY_SIDES
+    s = len(sides) - 1
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    nq, L = off[s + 1] - off[s], off[s + 1]
+    q = _dev(d["q"][:, :, off[s]:off[s + 1]], device)
+    k = _dev(d["k"][:, :, :L], device)
+    v = _dev(d["v"][:, :, :L], device)
+    del d
+    out = torch.empty_like(q)
+    dense = 4 * nq * L * D * B * H
+    res = []
+    for block in (128, 64):
+        cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, 5, 2, 4, block, block, device=device)
+        f, _ = kept_flops(cnt, idx, nq, L, block, D)
+        f *= B * H
+        ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, block, block, out=out),
+                     reps, device)
+        res.append({"granularity": f"block{block}", "density": f / dense, "ms": ms,
+                    "tflops": f / (ms * 1e-3) / 1e12})
+    cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, 5, 2, 4, 128, 128, device=device)
+    f, _ = kept_flops(cnt, idx, nq, L, 128, D)
+    f *= B * H
+    ms = time_ms(lambda: ops.sparvar_csla_token_attn_fwd(q, k, v, sides, s, 5, 2, 4, cnt, idx, out=out),
+                 reps, device)
+    res.append({"granularity": "token mask inside 128x128 tiles", "tile_density": f / dense, "ms": ms,
+                "tile_tflops": f / (ms * 1e-3) / 1e12})
+    return {"workload": "infinity2b_last_scale_csla_granularity", "B": B, "H": H, "D": D,
+            "mask": "csla sink<=5 r_prev=2 r_own=4", "runs": res}
 
 
 def density_sweep(device, reps=10, seed=0, B=2, H=16, D=128, densities=(0.05, 0.1, 0.2, 0.35, 0.5, 1.0)):
