@@ -12,6 +12,7 @@ import torch
 
 from block_sparse_cross_sparvar_b200 import inputs, ops
 from oracle import sparvar_oracle as orc
+from tests.selection_check import mass_selection_error
 
 pytestmark = pytest.mark.gpu
 
@@ -88,13 +89,18 @@ def test_cs4a_full_pass_every_scale():
                                              k_all[:, :, :off[dec + 1]], 0.95, lse=lse,
                                              return_mass=True)
     dcn, din, massn = dc.cpu().numpy(), di.cpu().numpy(), mass.cpu().numpy()
-    for b, h in pairs:
-        oc, oi, _, M, margin = orc.decide_blocks(_f(d["q"][b, h, off[dec]:off[dec + 1]]),
-                                                 _f(d["k"][b, h, :off[dec + 1]]), 128, 128, 0.95)
-        assert np.abs(massn[b, h] - M).max() < 2e-5
-        for qb in range(M.shape[0]):
-            if margin[qb] > 1e-4:
-                assert dcn[b, h, qb] == oc[qb] and np.array_equal(din[b, h, qb], oi[qb])
+    # the decision of every (batch, head) pair: masses against the oracle's; every row a
+    # valid selection of the kernel's own masses; beyond the margin the oracle's exact list
+    for b in range(B):
+        for h in range(H):
+            oc, oi, _, M, margin = orc.decide_blocks(_f(d["q"][b, h, off[dec]:off[dec + 1]]),
+                                                     _f(d["k"][b, h, :off[dec + 1]]), 128, 128, 0.95)
+            assert np.abs(massn[b, h] - M).max() < 2e-5
+            for qb in range(M.shape[0]):
+                err = mass_selection_error(dcn[b, h, qb], din[b, h, qb], massn[b, h, qb], 0.95)
+                assert err == "", (b, h, qb, err)
+                if margin[qb] > 1e-4:
+                    assert dcn[b, h, qb] == oc[qb] and np.array_equal(din[b, h, qb], oi[qb])
     src_nq, src_lkv = off[dec + 1] - off[dec], off[dec + 1]
     for s in range(dec + 1, len(INF)):
         nq, L = off[s + 1] - off[s], off[s + 1]
