@@ -359,14 +359,26 @@ int sparvar_wait_timeout_probe(uint64_t limit_ns, int32_t* dev_status, int32_t* 
   return SPARVAR_OK;
 }
 
-static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                         int H, int Lq, int Lkv, int D, const int64_t* q_strides,
-                         const int64_t* k_strides, const int64_t* v_strides,
-                         const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
-                         const int64_t* list_strides, int idx_row_len, const uint64_t* tile_mask,
-                         int mask_block, int block_q, int block_kv, float softmax_scale,
-                         int32_t* dev_status, void* stream,
-                         const sparvar::fwd::CslaTokens* tok) {
+// A checked single-problem launch of attn_fwd_kernel: arguments, tensor maps.
+struct FwdLaunch {
+  sparvar::fwd::Args a;
+  CUtensorMap tq, tk, tv;
+  sparvar::fwd::OutMaps to;
+  int D;
+  bool tok;
+};
+
+// Checks every argument of a single-problem attention call and encodes its tensor
+// maps; enqueues nothing.
+static int attn_fwd_prepare(FwdLaunch* L, const void* q, const void* k, const void* v, void* o,
+                            float* lse, int B, int H, int Lq, int Lkv, int D,
+                            const int64_t* q_strides, const int64_t* k_strides,
+                            const int64_t* v_strides, const int64_t* o_strides,
+                            const int32_t* kv_cnt, const int32_t* kv_idx,
+                            const int64_t* list_strides, int idx_row_len,
+                            const uint64_t* tile_mask, int mask_block, int block_q, int block_kv,
+                            float softmax_scale, int32_t* dev_status,
+                            const sparvar::fwd::CslaTokens* tok) {
   if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
   if (block_q != 128 || block_kv != 128)
     return fail(SPARVAR_ERR_UNSUPPORTED,
@@ -397,7 +409,8 @@ static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, f
   if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f))
     return fail(SPARVAR_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
 
-  sparvar::fwd::Args a{};
+  *L = FwdLaunch{};
+  sparvar::fwd::Args& a = L->a;
   a.B = B; a.H = H; a.n_problems = 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   sparvar::fwd::Problem& pr = a.prob[0];
@@ -418,20 +431,83 @@ static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, f
   a.dev_status = dev_status;
   if (tok) a.tok = *tok;
 
-  CUtensorMap tq, tk, tv;
-  sparvar::fwd::OutMaps to{};
-  if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
-  if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
-  if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
-  if ((rc = make_tmap(&to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o")))
+  if ((rc = make_tmap(&L->tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q")))
     return rc;
+  if ((rc = make_tmap(&L->tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k")))
+    return rc;
+  if ((rc = make_tmap(&L->tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v")))
+    return rc;
+  if ((rc = make_tmap(&L->to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o")))
+    return rc;
+  L->D = D;
+  L->tok = tok != nullptr;
+  return SPARVAR_OK;
+}
+
+static int attn_fwd_launch(const FwdLaunch& L, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tok) {
-    if (D == 128) return launch_fwd_kernel<128, true, false>(tq, tk, tv, to, a, st);
-    return launch_fwd_kernel<64, true, false>(tq, tk, tv, to, a, st);
+  if (L.tok) {
+    if (L.D == 128) return launch_fwd_kernel<128, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+    return launch_fwd_kernel<64, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
   }
-  if (D == 128) return launch_fwd_kernel<128, false, false>(tq, tk, tv, to, a, st);
-  return launch_fwd_kernel<64, false, false>(tq, tk, tv, to, a, st);
+  if (L.D == 128) return launch_fwd_kernel<128, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+  return launch_fwd_kernel<64, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+}
+
+// Device address of g_static_scratch in the current context.  Looked up with
+// cudaGetSymbolAddress once per (device, context) and cached: a new primary context
+// (after cudaDeviceReset) loads the module again, possibly elsewhere, so the cache
+// is keyed on the context as well as the device.
+using PFN_ctx_get_current = CUresult (*)(CUcontext*);
+static int static_scratch_address(void** out) {
+  static std::mutex mu;
+  static PFN_ctx_get_current get_ctx = nullptr;
+  static CUcontext ctx_of[128] = {};
+  static void* addr_of[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return fail(SPARVAR_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!get_ctx) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || !fn)
+      return fail(SPARVAR_ERR_CUDA, "cuCtxGetCurrent unavailable");
+    get_ctx = reinterpret_cast<PFN_ctx_get_current>(fn);
+  }
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (!ctx || ctx_of[dev] != ctx || !addr_of[dev]) {
+    // the lookup also binds the device's primary context when none is current yet
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+      return fail(SPARVAR_ERR_CUDA, "no current CUDA context");
+    ctx_of[dev] = ctx;
+    addr_of[dev] = a;
+  }
+  *out = addr_of[dev];
+  return SPARVAR_OK;
+}
+
+static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Lq, int Lkv, int D, const int64_t* q_strides,
+                         const int64_t* k_strides, const int64_t* v_strides,
+                         const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
+                         const int64_t* list_strides, int idx_row_len, const uint64_t* tile_mask,
+                         int mask_block, int block_q, int block_kv, float softmax_scale,
+                         int32_t* dev_status, void* stream,
+                         const sparvar::fwd::CslaTokens* tok) {
+  FwdLaunch L;
+  int rc = attn_fwd_prepare(&L, q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides,
+                            v_strides, o_strides, kv_cnt, kv_idx, list_strides, idx_row_len,
+                            tile_mask, mask_block, block_q, block_kv, softmax_scale, dev_status,
+                            tok);
+  if (rc) return rc;
+  return attn_fwd_launch(L, stream);
 }
 
 int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
@@ -659,6 +735,9 @@ int sparvar_block_sparse_attn_fwd_static(
   if (!list_strides) return fail(SPARVAR_ERR_INVALID_ARG, "list_strides is NULL");
   if (list_strides[0] < 0 || list_strides[1] < 0)
     return fail(SPARVAR_ERR_INVALID_ARG, "list strides must be >= 0");
+  if (idx_row_len < 0) return fail(SPARVAR_ERR_INVALID_ARG, "idx_row_len < 0");
+  if (ceil_div(Lkv, 128) > 4096)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "Lkv=%d gives more than 4096 KV tiles", Lkv);
   // tile counts, tile lists and tile masks, each 256-byte aligned, as sparvar_coarsen_lists
   // writes them
   const int64_t Bo = list_strides[0] == 0 ? 1 : B, Ho = list_strides[1] == 0 ? 1 : H;
@@ -671,37 +750,30 @@ int sparvar_block_sparse_attn_fwd_static(
     return fail(SPARVAR_ERR_UNSUPPORTED,
                 "tile lists need %lld bytes, the static scratch holds %zu",
                 static_cast<long long>(need), kStaticScratchBytes);
-  // the array's device address, looked up once per device
-  static std::mutex mu;
-  static void* addr[128] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 128) return fail(SPARVAR_ERR_UNSUPPORTED, "device %d", dev);
+  const int64_t t_strides[2] = {Bo > 1 ? Ho * nqt : 0, Ho > 1 ? nqt : 0};
+  // every argument of the attention launch is checked (on the host) before the scratch
+  // is looked up or the coarsening enqueued, so a refused call touches neither the
+  // scratch nor dev_status; the tile-list pointers are filled in afterwards
+  FwdLaunch L;
+  int rc = attn_fwd_prepare(&L, q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides,
+                            v_strides, o_strides, kv_cnt, kv_idx, t_strides,
+                            static_cast<int>(nkt), reinterpret_cast<const uint64_t*>(kv_idx),
+                            block, 128, 128, softmax_scale, dev_status, nullptr);
+  if (rc) return rc;
   void* base = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-      e = cudaGetSymbolAddress(&addr[dev], g_static_scratch);
-      if (e != cudaSuccess) {
-        addr[dev] = nullptr;
-        return cuda_fail(e, "cudaGetSymbolAddress");
-      }
-    }
-    base = addr[dev];
-  }
+  rc = static_scratch_address(&base);
+  if (rc) return rc;
   uint8_t* p = static_cast<uint8_t*>(base);
   int32_t* t_cnt = reinterpret_cast<int32_t*>(p);
   int32_t* t_idx = reinterpret_cast<int32_t*>(p + cnt_bytes);
   uint64_t* t_mask = reinterpret_cast<uint64_t*>(p + cnt_bytes + idx_bytes);
-  int rc = sparvar_coarsen_lists(kv_cnt, kv_idx, list_strides, idx_row_len, B, H, Lq, Lkv, block,
-                                 t_cnt, t_idx, t_mask, dev_status, stream);
+  L.a.prob[0].kv_cnt = t_cnt;
+  L.a.prob[0].kv_idx = t_idx;
+  L.a.tile_mask = t_mask;
+  rc = sparvar_coarsen_lists(kv_cnt, kv_idx, list_strides, idx_row_len, B, H, Lq, Lkv, block,
+                             t_cnt, t_idx, t_mask, dev_status, stream);
   if (rc) return rc;
-  const int64_t t_strides[2] = {Bo > 1 ? Ho * nqt : 0, Ho > 1 ? nqt : 0};
-  return sparvar_block_sparse_attn_fwd(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides,
-                                       v_strides, o_strides, t_cnt, t_idx, t_strides,
-                                       static_cast<int>(nkt), t_mask, block, 128, 128,
-                                       softmax_scale, dev_status, stream);
+  return attn_fwd_launch(L, stream);
 }
 
 }  // extern "C"

@@ -215,19 +215,27 @@ def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv
 def sparvar_block_sparse_attn_fwd_static(q, k, v, kv_cnt, kv_idx, block, softmax_scale=None,
                                          out=None, return_lse=False, dev_status=None):
     """Fine-grid (16/32/64) attention whose tile lists live in the library's static
-    device scratch: the only allocations here are the outputs, made by torch."""
+    device scratch: the only allocations here are the outputs, made by torch.
+
+    The lists are checked first: the C call cannot see their shapes, and lists
+    built for another block size would make the coarsening read past their end."""
     B, H, Lq, D = q.shape
     Lkv = k.shape[2]
+    if block not in (16, 32, 64):
+        raise SparvarError(f"block={block} not in (16, 32, 64)")
+    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32:
+        raise SparvarError("kv_cnt/kv_idx must be int32")
+    if kv_idx.shape[:-1] != kv_cnt.shape or not kv_idx.is_contiguous():
+        raise SparvarError("kv_idx must be contiguous with shape (*kv_cnt.shape, row_len)")
+    if kv_cnt.shape[-1] != -(-Lq // block):
+        raise SparvarError(f"kv_cnt has {kv_cnt.shape[-1]} query blocks, expected "
+                           f"{-(-Lq // block)} for block={block}")
     if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
         raise SparvarError("k/v must be [B, H, Lkv, D] matching q")
     qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
     if out is None:
         out = torch.empty_like(q, memory_format=torch.contiguous_format)
     os_ = _bhrd(out, "out")
-    if kv_cnt.dtype != torch.int32 or kv_idx.dtype != torch.int32:
-        raise SparvarError("kv_cnt/kv_idx must be int32")
-    if kv_idx.shape[:-1] != kv_cnt.shape or not kv_idx.is_contiguous():
-        raise SparvarError("kv_idx must be contiguous with shape (*kv_cnt.shape, row_len)")
     lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     sb, sh = _list_strides(kv_cnt, B, H)

@@ -1,7 +1,10 @@
 """The allocation-free fine-grid attention entry point (tile lists in the
-library's static device scratch) against the allocating path, which coarsens
-into caller buffers.  Collected last, so it also runs after every other test
-has used the library."""
+library's static device scratch) against the CPU fp64 oracle and against the
+allocating path, which coarsens into caller buffers.  It serves callers that
+may not allocate device memory (for instance a host that hands the library
+pre-sized buffers from its own pool and forbids cudaMalloc while its steps
+run).  Collected last, so it also runs after every other test has used the
+library."""
 import ctypes
 
 import numpy as np
@@ -9,6 +12,9 @@ import pytest
 import torch
 
 from block_sparse_cross_sparvar_b200 import build, inputs, ops
+from oracle import sparvar_oracle as orc
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
 
 
 def _lists(rng, B, H, nqb, nkb, p):
@@ -49,6 +55,20 @@ def test_static_scratch_matches_allocating_path_two_calls_in_a_row():
     torch.cuda.synchronize()
     for t, cnt, idx, block, o_s, lse_s, st in outs:
         assert st.item() == 0
+        # against the oracle: fp64 attention under the fine block mask, every row
+        B, H, Lq, D = t["q"].shape
+        nkb = -(-t["k"].shape[2] // block)
+        f = lambda x, b, h: x[b, h].double().cpu().numpy()  # noqa: E731
+        for b in range(B):
+            for h in range(H):
+                blk = orc.lists_to_blocks(cnt[b, h].cpu().numpy(), idx[b, h].cpu().numpy(), nkb)
+                O, L = orc.masked_attention(f(t["q"], b, h), f(t["k"], b, h), f(t["v"], b, h), blk,
+                                            block, block)
+                err = np.abs(o_s[b, h].double().cpu().numpy() - O)
+                assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (b, h, err.max())
+                got = lse_s[b, h].double().cpu().numpy()
+                assert np.array_equal(np.isfinite(got), np.isfinite(L))
+                assert np.abs(got[np.isfinite(L)] - L[np.isfinite(L)]).max() < 1e-3
         o_a, lse_a = ops.sparvar_block_sparse_attn_fwd(t["q"], t["k"], t["v"], cnt, idx, block,
                                                        block, return_lse=True)
         torch.cuda.synchronize()
@@ -73,6 +93,14 @@ def test_static_scratch_shared_lists():
     torch.cuda.synchronize()
     diff = (o_s.float() - o_a.float()).abs()
     assert diff.max().item() <= 1e-2 and diff.mean().item() <= 1e-5
+    _, _, blk = orc.build_csla_mask(inputs.TINY_SIDES, 4, 2, 1, 1, 16, 16)
+    f = lambda bits, b, h: (bits[b, h].astype(np.uint32) << 16).view(np.float32).astype(np.float64)  # noqa: E731
+    for b in range(2):
+        for h in range(2):
+            O, _ = orc.masked_attention(f(d["q"][:, :, off[4]:off[5]], b, h), f(d["k"], b, h),
+                                        f(d["v"], b, h), blk, 16, 16)
+            err = np.abs(o_s[b, h].double().cpu().numpy() - O)
+            assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
 
 
 def test_static_scratch_rejects_oversize_and_bad_blocks_on_host():
@@ -94,3 +122,31 @@ def test_static_scratch_rejects_oversize_and_bad_blocks_on_host():
     assert call(block=8) == 2
     assert call(Lq=0) == 1
     assert call(ls=(-1, 0)) == 1
+
+    # an attention argument the kernel cannot take (D = 96) is refused on the host,
+    # before the scratch is looked up or the coarsening enqueued
+    def call_d(D):
+        return lib.sparvar_block_sparse_attn_fwd_static(
+            vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 128, 128, D, i64(0, 0, 128),
+            i64(0, 0, 128), i64(0, 0, 128), i64(0, 0, 128), vp(16), vp(16), i64(1, 1), 8, 16,
+            0.1, vp(0), vp(0))
+    assert call_d(96) == 2 and "D=96" in lib.sparvar_last_error().decode()
+    # a bad stride of q is refused the same way
+    assert lib.sparvar_block_sparse_attn_fwd_static(
+        vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 128, 128, 128, i64(0, 0, 100),
+        i64(0, 0, 128), i64(0, 0, 128), i64(0, 0, 128), vp(16), vp(16), i64(1, 1), 8, 16, 0.1,
+        vp(0), vp(0)) == 1
+
+
+def test_static_binding_refuses_lists_of_another_block_size():
+    """Lists built over 64-token blocks passed with block=16 would make the coarsening
+    read past the end of kv_cnt and kv_idx: the binding refuses them before any call."""
+    Lq, Lkv, D = 300, 777, 64
+    q = torch.zeros(1, 1, Lq, D, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, Lkv, D, dtype=torch.bfloat16)
+    cnt = torch.ones(-(-Lq // 64), dtype=torch.int32)
+    idx = torch.zeros(-(-Lq // 64), -(-Lkv // 64), dtype=torch.int32)
+    with pytest.raises(ops.SparvarError, match="query blocks"):
+        ops.sparvar_block_sparse_attn_fwd_static(q, k, k, cnt, idx, 16)
+    with pytest.raises(ops.SparvarError, match="block=128"):
+        ops.sparvar_block_sparse_attn_fwd_static(q, k, k, cnt, idx, 128)
