@@ -44,22 +44,38 @@ def peaks():
 
 
 def profiled_traffic():
-    """DRAM bytes per launch of the attention kernel from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
+    """DRAM bytes per launch of the attention kernel from the committed ncu data
+    file, if it was taken on the current kernel source (else None)."""
     import hashlib
     try:
         src = os.path.join(ROOT, "block_sparse_cross_sparvar_b200", "csrc", "attn_fwd_kernel.cuh")
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        fields = {}
-        for line in open(os.path.join(ROOT, "profiles", "attn_fwd_infinity2b_last.md")):
-            if ":" in line and not line.startswith("|"):
-                key, _, val = line.partition(":")
-                fields[key.strip()] = val.strip()
-        if fields.get("kernel_source_sha256_16") == sha:
-            return int(fields["traffic_bytes_per_launch"])
+        with open(os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")) as f:
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256_16") == sha:
+            return int(rec["traffic_bytes_per_launch"])
     except Exception:
         pass
     return None
+
+
+def workload_config(wl, cnt, idx, world):
+    """The ``config`` object of the JSON line, identical for both arms: the
+    workload, its shapes and the kept blocks of its CSLA lists."""
+    sides, k, bq, D = wl["sides"], wl["q_scale"], wl["block"], wl["D"]
+    off = inputs.token_offsets(sides)
+    nq, L = off[k + 1] - off[k], off[k + 1]
+    flops = kept_flops_from_lists(cnt, idx, nq, L, bq, bq, D) * wl["B"] * wl["H"]
+    dense = 4 * nq * L * D * wl["B"] * wl["H"]
+    return {"workload": wl["name"], "B": wl["B"], "H": wl["H"], "Lq": nq, "Lkv": L, "D": D,
+            "block_q": bq, "block_kv": bq,
+            "mask": f"csla sink<={wl['n_sink_scales']} r_prev={wl['radius_prev']} "
+                    f"r_own={wl['radius_own']}",
+            "kept_blocks": int(np.asarray(cnt).sum()), "total_blocks": int(idx.shape[0] * idx.shape[1]),
+            "kept_flop_fraction": flops / dense,
+            "kept_gflop_per_step_per_gpu": flops / 1e9,
+            "l2": "256 MB flush write between timed steps",
+            "parallelism": f"independent batch per GPU x{world}"}
 
 
 def kept_flops_from_lists(cnt, idx, nq, L, bq, bk, D):
@@ -160,8 +176,11 @@ def cpu_baseline(wl, budget_s=12.0, seed=0, d=None):
 def run_reference(args, wl, rank, world):
     if world > 1 and rank != 0:
         return
+    from oracle import sparvar_oracle as orc
     per_step = []
     d = inputs.make_qkv(0, wl["B"], wl["H"], wl["sides"], wl["D"], wl["n_sink_scales"])
+    cnt, idx, _ = orc.build_csla_mask(wl["sides"], wl["q_scale"], wl["n_sink_scales"],
+                                      wl["radius_prev"], wl["radius_own"], wl["block"], wl["block"])
     budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         res = cpu_baseline(wl, budget_s=budget, d=d)
@@ -173,9 +192,7 @@ def run_reference(args, wl, rank, world):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": float(np.mean([r["seconds"] for r in per_step]) * 1e3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl["name"], "B": wl["B"], "H": wl["H"],
-                                            "Lq": 4096, "Lkv": 10521, "D": wl["D"],
-                                            "block": wl["block"], "mask": "csla"},
+            "data": "synthetic", "config": workload_config(wl, cnt, idx, world),
             "cpu_baseline": {k: per_step[-1][k] for k in ("kind", "cores", "sample")} | {"value": val,
                                                                                       "unit": "TFLOP/s"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -242,8 +259,6 @@ def main():
     torch.cuda.synchronize()
     cnt_h, idx_h = cnt.cpu().numpy(), idx.cpu().numpy()
     flops_step = kept_flops_from_lists(cnt_h, idx_h, nq, L, bq, bq, D) * B * H
-    dense_flops = 4 * nq * L * D * B * H
-    nqb, nkb = idx_h.shape
 
     for _ in range(args.warmup):
         step(q, kk, vv, o)
@@ -319,20 +334,14 @@ def main():
             "attn_ms": t_attn, "mask_build_ms": float(np.mean(mask_ms)),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl["name"], "B": B, "H": H, "Lq": nq, "Lkv": L, "D": D,
-                       "block_q": bq, "block_kv": bq, "mask": "csla sink<=5 r_prev=2 r_own=4",
-                       "kept_blocks": int(cnt_h.sum()), "total_blocks": int(nqb * nkb),
-                       "kept_flop_fraction": flops_step / dense_flops,
-                       "kept_gflop_per_step_per_gpu": flops_step / 1e9,
-                       "l2": "256 MB flush write between timed steps",
-                       "parallelism": f"independent batch per GPU x{world}"},
+            "config": workload_config(wl, cnt_h, idx_h, world),
             "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128, TOK=false, MULTI=false>",
                          "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16"],
                          "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']}",
                          "traffic": profiled_traffic(),
-                         "traffic_note": "ncu dram bytes read+write per launch (profiles/attn_fwd_infinity2b_last.md); "
-                                         "null when the kernel source changed since"},
+                         "traffic_note": "ncu dram bytes read+write per launch of this kernel source; "
+                                         "null when the source changed since the capture"},
             "e2e": {"value": total_flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": t_e2e,
                     "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
