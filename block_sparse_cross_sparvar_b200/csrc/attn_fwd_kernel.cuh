@@ -69,9 +69,6 @@ constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
 constexpr uint64_t kDrainNs = 500000000ull;   // 0.5 s per drain
 constexpr int kMaxSlots = 12;
 constexpr int kRel = 16;                      // release barriers (more than ring slots)
-// Of each 16 pairs of score columns, those whose bit is set take the FMA-pipe 2^x
-// (exp2_poly2), the others the MUFU ex2.
-constexpr uint32_t kPolyPairs = 0x0u;
 
 // CSLA token mask applied inside the kept tiles (enabled != 0): the query scale,
 // the sink length in tokens and the locality radii over the schedule.
@@ -614,8 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
         // pass 2: P = 2^(s * scale - m) in packed pairs.  Columns 96-127 are re-read
         // while the columns held in registers are worked on; P chunk cc (packed bf16)
-        // overwrites TMEM columns [16cc, 16cc + 16), already read.  The pairs
-        // kPolyPairs selects take the FMA-pipe exponential, the others the MUFU one.
+        // overwrites TMEM columns [16cc, 16cc + 16), already read.
         const uint64_t sc2 = f2_pack(csc, csc), neg2 = f2_pack(neg, neg);
         uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
         auto p_chunk = [&](const uint32_t(&cur)[32], int cc) {
@@ -626,12 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(f2_fma(f2_pack(__uint_as_float(cur[2 * k]), __uint_as_float(cur[2 * k + 1])),
                              sc2, neg2),
                       e0, e1);
-            if ((kPolyPairs >> k) & 1u) {
-              exp2_poly2(e0, e1, p0, p1);
-            } else {
-              p0 = ex2_approx(e0);
-              p1 = ex2_approx(e1);
-            }
+            p0 = ex2_approx(e0);
+            p1 = ex2_approx(e1);
             if (k & 1) {
               acc1 = f2_add(acc1, f2_pack(p0, p1));
             } else {

@@ -233,45 +233,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 2^x for two values on the FMA and integer pipes, leaving the MUFU unit to
-// other elements.  Range reduction: x = j + f with j the nearest integer
-// (adding 1.5 * 2^23 in round-to-nearest leaves j in the low mantissa bits) and
-// |f| <= 1/2; then 2^f ~ p(f) = 1 + c1 f + c2 f^2 + c3 f^3 and 2^j is added
-// into the exponent field.  The cubic minimises the maximum relative error on
-// [-1/2, 1/2] with the constant term held at 1 (weighted least squares with
-// Lawson's reweighting): 1.0e-4 in fp32 Horner form, against bf16's rounding
-// step of 2^-9.  Inputs are first clamped to -127, where j = -127, f = 0 and
-// p = 1 give exactly +0 (so -inf maps to 0); inputs must be below 128.
-constexpr float kExp2C1 = 0.69328296f;
-constexpr float kExp2C2 = 0.242211f;
-constexpr float kExp2C3 = 0.055008914f;
-constexpr float kExp2Shift = 12582912.0f;  // 1.5 * 2^23
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t shift = f2_pack(kExp2Shift, kExp2Shift);
-  const uint64_t xc = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const uint64_t t = f2_add(xc, shift);          // j in the low bits
-  const uint64_t f = f2_sub(xc, f2_sub(t, shift));
-  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(1.f, 1.f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt packs its first source into the upper half.

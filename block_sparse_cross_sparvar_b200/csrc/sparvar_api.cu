@@ -14,7 +14,7 @@
 
 #include "../../include/sparvar.h"
 #include "attn_fwd_kernel.cuh"
-#include "attn_kernel.cuh"
+#include "decide_kernel.cuh"
 #include "mask_kernels.cuh"
 #include "ocache_kernel.cuh"
 #include "wait_probe_kernel.cuh"
@@ -125,18 +125,18 @@ int check_operand(const void* p, const int64_t* st, int B, int H, int rows, int 
   return SPARVAR_OK;
 }
 
-template <int D, int MODE>
-int launch_attn_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const sparvar::AttnArgs& a, cudaStream_t stream) {
-  auto kern = sparvar::block_sparse_attn_kernel<D, MODE>;
-  const uint32_t smem = sparvar::Smem<D>::dyn_bytes(MODE);
+template <int D>
+int launch_decide_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const sparvar::DecideArgs& a,
+                         cudaStream_t stream) {
+  auto kern = sparvar::decide_blocks_kernel<D>;
+  const uint32_t smem = sparvar::Smem<D>::dyn_bytes();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   dim3 grid(a.nqb, a.H, a.B);
-  kern<<<grid, sparvar::kThreads, smem, stream>>>(tq, tk, tv, a);
+  kern<<<grid, sparvar::kThreads, smem, stream>>>(tq, tk, a);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "block_sparse_attn_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "decide_blocks_kernel launch");
   return SPARVAR_OK;
 }
 
@@ -659,7 +659,7 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   if (!(topk_ratio >= 0.f && topk_ratio <= 1.f))
     return fail(SPARVAR_ERR_INVALID_ARG, "topk_ratio must be in [0, 1] (0: mass threshold)");
 
-  sparvar::AttnArgs a{};
+  sparvar::DecideArgs a{};
   a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
   a.nqb = static_cast<int>(ceil_div(Lq, 128));
   a.nkb = nkb;
@@ -677,8 +677,8 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
   if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_attn_kernel<128, sparvar::kModeMass>(tq, tk, tk, a, st);
-  return launch_attn_kernel<64, sparvar::kModeMass>(tq, tk, tk, a, st);
+  if (D == 128) return launch_decide_kernel<128>(tq, tk, a, st);
+  return launch_decide_kernel<64>(tq, tk, a, st);
 }
 
 int sparvar_ocache_apply(const void* o_target, const void* o_dense, const void* o_sparse, void* out,
