@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsparvar.so")
 SOURCES = ["sparvar_api.cu"]
-HEADERS = ["attn_fwd_kernel.cuh", "decide_kernel.cuh", "mask_kernels.cuh", "ocache_kernel.cuh", "ptx.cuh",
+HEADERS = ["attn_fwd_kernel.cuh", "decide_kernel.cuh", "mask_kernels.cuh", "ocache_kernel.cuh", "ptx.cuh", "select.cuh",
            "tmem_io.cuh", "wait_probe_kernel.cuh"]
 
 

@@ -22,6 +22,7 @@
 #include <cuda.h>
 
 #include "ptx.cuh"
+#include "select.cuh"
 #include "tmem_io.cuh"
 
 namespace sparvar {
@@ -262,52 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("bar.sync 1, 128;" ::: "memory");
     const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
     if (warp == 0 && !aborted && good) {
-      const int nkb = args.nkb;
-      const int nq_blk = min(kTile, args.Lq - qb * kTile);
-      const float inv_nq = 1.f / static_cast<float>(nq_blk);
       const int64_t rowid = (static_cast<int64_t>(b) * args.H + h) * args.nqb + qb;
-      for (int i = lane; i < nkb; i += 32) {
-        const float mval = mass_sh[i] * inv_nq;
-        mass_sh[i] = mval;
-        if (args.mass_out) args.mass_out[rowid * nkb + i] = mval;
-      }
-      __syncwarp();
-      float run = 0.f;
-      int taken = 0;
-      const int limit = args.topk > 0 ? min(args.topk, nkb) : nkb;
-      while (taken < limit) {
-        float best = -1.f;
-        int best_i = 0x7fffffff;
-        for (int i = lane; i < nkb; i += 32) {
-          if (!kept_sh[i]) {
-            const float mv = mass_sh[i];
-            if (mv > best || (mv == best && i < best_i)) { best = mv; best_i = i; }
-          }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
-          if (ob > best || (ob == best && oi < best_i)) { best = ob; best_i = oi; }
-        }
-        if (lane == 0) kept_sh[best_i] = 1;
-        __syncwarp();
-        run += best;
-        ++taken;
-        if (args.topk <= 0 && run >= args.mass_threshold) break;
-      }
-      // ascending compaction
-      int base = 0;
-      int32_t* out = args.sel_idx + rowid * nkb;
-      for (int i0 = 0; i0 < nkb; i0 += 32) {
-        const int i = i0 + lane;
-        const bool k = i < nkb && kept_sh[i];
-        const uint32_t bal = __ballot_sync(0xffffffffu, k);
-        if (k) out[base + __popc(bal & ((1u << lane) - 1u))] = i;
-        base += __popc(bal);
-      }
-      for (int i = base + lane; i < nkb; i += 32) out[i] = -1;
-      if (lane == 0) args.sel_cnt[rowid] = base;
+      select_blocks_warp(mass_sh, kept_sh, args.nkb, min(kTile, args.Lq - qb * kTile), args.topk,
+                         args.mass_threshold,
+                         args.mass_out ? args.mass_out + rowid * args.nkb : nullptr,
+                         args.sel_idx + rowid * args.nkb, args.sel_cnt + rowid);
     }
   }
 

@@ -80,10 +80,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 4-D map over a [B][H][rows][D] bf16 tensor: box = 64 columns x 128 rows,
-// 128-byte swizzle, zero fill outside the tensor.
+// 4-D map over a [B][H][rows][D] bf16 tensor: box = 64 columns x box_rows rows
+// (128 for loads, one warp's 32 rows for the attention output), 128-byte swizzle,
+// zero fill outside the tensor.
 int make_tmap(CUtensorMap* m, const void* base, int D, int rows, int H, int B, int64_t sr,
-              int64_t sh, int64_t sb, const char* name) {
+              int64_t sh, int64_t sb, const char* name, int box_rows = 128) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(SPARVAR_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   if (H == 1) sh = static_cast<int64_t>(rows) * sr;
@@ -92,7 +93,7 @@ int make_tmap(CUtensorMap* m, const void* base, int D, int rows, int H, int B, i
                         static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(sr * 2), static_cast<cuuint64_t>(sh * 2),
                            static_cast<cuuint64_t>(sb * 2)};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -140,28 +141,37 @@ int launch_decide_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const spa
   return SPARVAR_OK;
 }
 
-template <int D, bool TOK, bool MULTI>
+template <int D, bool TOK, bool MULTI, bool DEC = false>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const sparvar::fwd::OutMaps& to, const sparvar::fwd::Args& a,
                       cudaStream_t stream) {
-  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI>;
+  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI, DEC>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-  // persistent: one CTA per SM, each walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  // the kernel's warpgroups trade registers (setmaxnreg) on the assumption that each
+  // thread was launched with exactly kLaunchRegs; any other count could leave a
+  // warpgroup waiting for registers that never come, so it is refused
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+  if (fa.numRegs != sparvar::fwd::kLaunchRegs)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "attn_fwd_kernel compiled with %d registers per thread, "
+                "its register budgets assume %d", fa.numRegs, sparvar::fwd::kLaunchRegs);
+  // persistent: one CTA per SM, claiming the pairs blockIdx.x, blockIdx.x + gridDim.x, ...
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
-  const int64_t tiles = a.total_tiles;
-  const int64_t grid = tiles < sms ? tiles : sms;
-  // the kernel's per-CTA sequence counters (blocks, ring positions) are 32-bit
+  const int64_t pairs = a.total_pairs;
+  const int64_t grid = pairs < sms ? pairs : sms;
+  // the kernel's per-CTA sequence counters (blocks, ring loads) are 32-bit
   int64_t row_len = 0;
   for (int i = 0; i < a.n_problems; ++i) row_len = std::max<int64_t>(row_len, a.prob[i].idx_row_len);
-  if (ceil_div(tiles, grid) * (3 * row_len + 1) >= (int64_t{1} << 31))
-    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %lld too large per SM",
-                static_cast<long long>(tiles), static_cast<long long>(row_len));
+  if (ceil_div(pairs, grid) * (8 * row_len + 8) >= (int64_t{1} << 31))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tile pairs x idx_row_len %lld too large per SM",
+                static_cast<long long>(pairs), static_cast<long long>(row_len));
   kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
@@ -417,11 +427,11 @@ static int attn_fwd_prepare(FwdLaunch* L, const void* q, const void* k, const vo
   pr.Lq = Lq; pr.Lkv = Lkv;
   pr.nqb = static_cast<int>(ceil_div(Lq, 128));
   pr.nkb = static_cast<int>(ceil_div(Lkv, 128));
-  pr.q_row0 = 0; pr.tile0 = 0;
+  pr.q_row0 = 0; pr.pair0 = 0;
   pr.kv_cnt = kv_cnt; pr.kv_idx = kv_idx;
   pr.list_sb = list_strides[0]; pr.list_sh = list_strides[1];
   pr.idx_row_len = idx_row_len;
-  a.total_tiles = static_cast<int>(static_cast<int64_t>(B) * H * pr.nqb);
+  a.total_pairs = static_cast<int>(static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2));
   a.tile_mask = tile_mask;
   a.mask_shift = mask_shift;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -437,7 +447,8 @@ static int attn_fwd_prepare(FwdLaunch* L, const void* q, const void* k, const vo
     return rc;
   if ((rc = make_tmap(&L->tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v")))
     return rc;
-  if ((rc = make_tmap(&L->to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o")))
+  if ((rc = make_tmap(&L->to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o",
+                      sparvar::fwd::kOutBoxRows)))
     return rc;
   L->D = D;
   L->tok = tok != nullptr;
@@ -551,7 +562,7 @@ int sparvar_block_sparse_attn_fwd_multi(
   sparvar::fwd::Args a{};
   a.B = B; a.H = H; a.n_problems = n_problems;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  int64_t tiles = 0;
+  int64_t pairs = 0;
   for (int i = 0; i < n_problems; ++i) {
     if (q_row0[i] < 0 || lq[i] < 1 || static_cast<int64_t>(q_row0[i]) + lq[i] > q_rows)
       return fail(SPARVAR_ERR_INVALID_ARG, "problem %d: query rows [%d, %d + %d) outside [0, %d)", i,
@@ -566,15 +577,15 @@ int sparvar_block_sparse_attn_fwd_multi(
     pr.nqb = static_cast<int>(ceil_div(lq[i], 128));
     pr.nkb = static_cast<int>(ceil_div(lkv[i], 128));
     pr.q_row0 = q_row0[i];
-    pr.tile0 = static_cast<int>(tiles);
+    pr.pair0 = static_cast<int>(pairs);
     pr.kv_cnt = kv_cnt[i]; pr.kv_idx = kv_idx[i];
     pr.list_sb = list_strides[2 * i]; pr.list_sh = list_strides[2 * i + 1];
     pr.idx_row_len = idx_row_len[i];
-    tiles += static_cast<int64_t>(B) * H * pr.nqb;
-    if (tiles > (int64_t{1} << 30))
-      return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
+    pairs += static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2);
+    if (pairs > (int64_t{1} << 30))
+      return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tile pairs");
   }
-  a.total_tiles = static_cast<int>(tiles);
+  a.total_pairs = static_cast<int>(pairs);
   a.tile_mask = nullptr;
   a.mask_shift = 7;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -595,7 +606,7 @@ int sparvar_block_sparse_attn_fwd_multi(
     // the problem's own rows only, so the last tile's rows past its end are clipped
     const void* base = static_cast<const __nv_bfloat16*>(o) + q_row0[i] * o_strides[2];
     if ((rc = make_tmap(&to.m[i], base, D, lq[i], H, B, o_strides[2], o_strides[1], o_strides[0],
-                        "o")))
+                        "o", sparvar::fwd::kOutBoxRows)))
       return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -679,6 +690,73 @@ int sparvar_decide_blocks(const void* q, const void* k, int B, int H, int Lq, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 128) return launch_decide_kernel<128>(tq, tk, a, st);
   return launch_decide_kernel<64>(tq, tk, a, st);
+}
+
+int sparvar_decision_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int Lq, int Lkv, int D, const int64_t* q_strides,
+                              const int64_t* k_strides, const int64_t* v_strides,
+                              const int64_t* o_strides, float softmax_scale, float mass_threshold,
+                              float topk_ratio, int32_t* kv_cnt, int32_t* kv_idx, float* mass,
+                              int32_t* dev_status, void* stream) {
+  if (D != 64 && D != 128) return fail(SPARVAR_ERR_UNSUPPORTED, "D=%d not in {64, 128}", D);
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
+    return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
+  const int nkb = static_cast<int>(ceil_div(Lkv, 128));
+  if (nkb > sparvar::fwd::kMaxDecBlocks)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "Lkv=%d gives %d KV blocks (max %d)", Lkv, nkb,
+                sparvar::fwd::kMaxDecBlocks);
+  if (static_cast<int64_t>(B) * H * ceil_div(Lq, 128) > (int64_t{1} << 30))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "B*H*ceil(Lq/128) above 2^30 query tiles");
+  int rc;
+  if ((rc = check_operand(q, q_strides, B, H, Lq, D, "q"))) return rc;
+  if ((rc = check_operand(k, k_strides, B, H, Lkv, D, "k"))) return rc;
+  if ((rc = check_operand(v, v_strides, B, H, Lkv, D, "v"))) return rc;
+  if ((rc = check_operand(o, o_strides, B, H, Lq, D, "o"))) return rc;
+  if (!kv_cnt || !kv_idx) return fail(SPARVAR_ERR_INVALID_ARG, "kv_cnt/kv_idx is NULL");
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f) || std::isnan(mass_threshold))
+    return fail(SPARVAR_ERR_INVALID_ARG,
+                "softmax_scale must be finite and > 0, mass_threshold a number");
+  if (!(topk_ratio >= 0.f && topk_ratio <= 1.f))
+    return fail(SPARVAR_ERR_INVALID_ARG, "topk_ratio must be in [0, 1] (0: mass threshold)");
+
+  sparvar::fwd::Args a{};
+  a.B = B; a.H = H; a.n_problems = 1;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  sparvar::fwd::Problem& pr = a.prob[0];
+  pr.Lq = Lq; pr.Lkv = Lkv;
+  pr.nqb = static_cast<int>(ceil_div(Lq, 128));
+  pr.nkb = nkb;
+  pr.q_row0 = 0; pr.pair0 = 0;
+  pr.idx_row_len = nkb;
+  a.total_pairs = static_cast<int>(static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2));
+  a.mask_shift = 7;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
+  a.lse = lse;
+  a.lse_rows = Lq;
+  a.dev_status = dev_status;
+  a.mass_out = mass;
+  a.mass_threshold = mass_threshold;
+  // k = ceil(ratio * NKB), at least one; the allowance keeps 0.2f * 20 at 4
+  a.topk = topk_ratio > 0.f
+               ? static_cast<int>(std::min<double>(
+                     nkb, std::max<double>(1.0, std::ceil(static_cast<double>(topk_ratio) * nkb - 1e-6))))
+               : 0;
+  a.sel_cnt = kv_cnt;
+  a.sel_idx = kv_idx;
+  CUtensorMap tq, tk, tv;
+  sparvar::fwd::OutMaps to{};
+  if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
+  if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
+  if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
+  if ((rc = make_tmap(&to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o",
+                      sparvar::fwd::kOutBoxRows)))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return launch_fwd_kernel<128, false, false, true>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64, false, false, true>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_ocache_apply(const void* o_target, const void* o_dense, const void* o_sparse, void* out,

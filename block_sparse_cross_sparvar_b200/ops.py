@@ -56,6 +56,8 @@ EXPORTS = {
                               _i),
     "sparvar_validate_lists": ([_vp, _vp, _i, _i, _i, _vp, _vp], _i),
     "sparvar_wait_timeout_probe": ([ctypes.c_uint64, _vp, _vp, _vp], _i),
+    "sparvar_decision_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p, _i64p,
+                                   _i64p, _f, _f, _f, _vp, _vp, _vp, _vp, _vp], _i),
 }
 
 
@@ -347,6 +349,34 @@ def sparvar_decide_blocks(q, k, mass_threshold, lse=None, softmax_scale=None, bl
         _ptr(dev_status),
         _stream(q.device)), "sparvar_decide_blocks")
     return cnt, idx, mass
+
+
+def sparvar_decision_attn_fwd(q, k, v, mass_threshold, topk_ratio=0.0, softmax_scale=None,
+                              out=None, return_mass=False, dev_status=None):
+    """Dense attention at the decision scale with the CS4A decision fused in.
+
+    Returns (O [B,H,Lq,D], LSE [B,H,Lq], kv_cnt [B,H,NQB], kv_idx [B,H,NQB,NKB],
+    mass [B,H,NQB,NKB] or None), 128 x 128 blocks."""
+    B, H, Lq, D = q.shape
+    Lkv = k.shape[2]
+    if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
+        raise SparvarError("k/v must be [B, H, Lkv, D] matching q")
+    qs, ks, vs = _bhrd(q, "q"), _bhrd(k, "k"), _bhrd(v, "v")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    os_ = _bhrd(out, "out")
+    nqb, nkb = -(-Lq // 128), -(-Lkv // 128)
+    dev = q.device
+    lse = torch.empty(B, H, Lq, dtype=torch.float32, device=dev)
+    cnt = torch.empty(B, H, nqb, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, H, nqb, nkb, dtype=torch.int32, device=dev)
+    mass = torch.empty(B, H, nqb, nkb, dtype=torch.float32, device=dev) if return_mass else None
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    _check(lib().sparvar_decision_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_, scale,
+        float(mass_threshold), float(topk_ratio), _ptr(cnt), _ptr(idx), _ptr(mass),
+        _ptr(dev_status), _stream(dev)), "sparvar_decision_attn_fwd")
+    return out, lse, cnt, idx, mass
 
 
 def sparvar_map_indices(src_cnt, src_idx, src_nq, src_lkv, dst_nq, dst_lkv, block_q=128,

@@ -122,7 +122,7 @@ def cs4a_topk_2d_pass(device, reps=10, seed=0):
 
 
 def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision_scale=9,
-                   topk_ratio=0.0, mapping="1d", ocache=False):
+                   topk_ratio=0.0, mapping="1d", ocache=False, fused_decision=True):
     sides = inputs.INFINITY_SIDES
     d = inputs.make_qkv(seed, B, H, sides, D, 5)
     off = d["offsets"]
@@ -141,7 +141,13 @@ def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision
             k = k_all[:, :, :off[s + 1]]
             v = v_all[:, :, :off[s + 1]]
             cnt, idx = dense[s]
-            if s == decision_scale:
+            if s == decision_scale and fused_decision:
+                _, _, dc, di, _ = ops.sparvar_decision_attn_fwd(q, k, v, tau, topk_ratio=topk_ratio,
+                                                                out=outs[s])
+                state["dec"] = (dc, di)
+                if ocache:
+                    state["o_sparse"] = ops.sparvar_block_sparse_attn_fwd(q, k, v, dc, di)
+            elif s == decision_scale:
                 _, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=outs[s], return_lse=True)
                 dc, di, _ = ops.sparvar_decide_blocks(q, k, tau, lse=lse, topk_ratio=topk_ratio)
                 state["dec"] = (dc, di)
@@ -178,10 +184,43 @@ def cs4a_full_pass(device, reps=10, seed=0, B=2, H=16, D=128, tau=0.95, decision
                                                 "density": f / (4 * nq * L * D * B * H)}
         flops += f
     rule = (f"topk {topk_ratio}" if topk_ratio > 0 else f"mass {tau}") + (" + ocache" if ocache else "")
+    rule += ", fused decision" if fused_decision else ", decision after the dense pass"
     return {"workload": f"cs4a_full_pass_13_scales_{mapping}_mapping", "B": B, "H": H, "D": D,
             "selection": rule,
             "ms": ms, "gflop": flops / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
             "scales": per_scale}
+
+
+def decision_fused_vs_separate(device, reps=20, seed=0, B=2, H=16, D=128, decision_scale=9):
+    """The decision scale (32x32 over its 2521-key prefix): dense attention with the
+    decision fused in (one launch) against dense attention followed by the
+    stand-alone decision kernel (two launches, QK^T recomputed), for the mass
+    rule and the Top-K rule."""
+    sides = inputs.INFINITY_SIDES
+    d = inputs.make_qkv(seed, B, H, sides, D, 5)
+    off = d["offsets"]
+    s = decision_scale
+    q = _dev(d["q"][:, :, off[s]:off[s + 1]], device)
+    k = _dev(d["k"][:, :, :off[s + 1]], device)
+    v = _dev(d["v"][:, :, :off[s + 1]], device)
+    del d
+    nq, L = off[s + 1] - off[s], off[s + 1]
+    cnt, idx = _dense_lists(-(-nq // 128), -(-L // 128), device)
+    out = torch.empty_like(q)
+    dense = 4 * nq * L * D * B * H
+    res = []
+    for tau, ratio in ((0.95, 0.0), (0.0, 0.2)):
+        def separate():
+            _, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=out, return_lse=True)
+            ops.sparvar_decide_blocks(q, k, tau, lse=lse, topk_ratio=ratio)
+
+        ms_sep = time_ms(separate, reps, device)
+        ms_fused = time_ms(lambda: ops.sparvar_decision_attn_fwd(q, k, v, tau, topk_ratio=ratio,
+                                                                 out=out), reps, device)
+        res.append({"selection": f"topk {ratio}" if ratio > 0 else f"mass {tau}",
+                    "fused_ms": ms_fused, "separate_ms": ms_sep,
+                    "dense_tflops_fused": dense / (ms_fused * 1e-3) / 1e12})
+    return {"workload": "cs4a_decision_scale_32x32", "B": B, "H": H, "D": D, "runs": res}
 
 
 def csla_radius_sweep(device, reps=10, seed=0, B=2, H=32, D=128, radii=(1, 2, 4)):
@@ -231,10 +270,24 @@ def csla_granularity_sweep(device, reps=10, seed=0, B=2, H=16, D=128):
         cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, 5, 2, 4, block, block, device=device)
         f, _ = kept_flops(cnt, idx, nq, L, block, D)
         f *= B * H
-        ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, block, block, out=out),
-                     reps, device)
-        res.append({"granularity": f"block{block}", "density": f / dense, "ms": ms,
-                    "tflops": f / (ms * 1e-3) / 1e12})
+        if block == 128:
+            ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=out), reps,
+                         device)
+            res.append({"granularity": "block128", "density": f / dense, "ms": ms,
+                        "tflops": f / (ms * 1e-3) / 1e12})
+            continue
+        # 64x64 lists: coarsened to 128x128 tiles with per-tile masks inside the
+        # allocation-free call (no allocation in the timed region; the coarsening
+        # kernel is timed with the attention); the executed tiles' work is reported too
+        ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd_static(q, k, v, cnt, idx, block,
+                                                                      out=out), reps, device)
+        t_cnt, t_idx, _ = ops.sparvar_coarsen_lists(cnt, idx, B, H, nq, L, block)
+        ft, _ = kept_flops(t_cnt.reshape(-1), t_idx.reshape(-1, t_idx.shape[-1]), nq, L, 128, D)
+        ft *= B * H
+        res.append({"granularity": "block64", "density": f / dense, "ms": ms,
+                    "tflops": f / (ms * 1e-3) / 1e12, "tile_density": ft / dense,
+                    "tile_tflops": ft / (ms * 1e-3) / 1e12,
+                    "note": "coarsening kernel included, no allocation in the timed region"})
     cnt, idx, _ = ops.sparvar_build_csla_mask(sides, s, 5, 2, 4, 128, 128, device=device)
     f, _ = kept_flops(cnt, idx, nq, L, 128, D)
     f *= B * H

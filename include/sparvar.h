@@ -139,6 +139,36 @@ SPARVAR_API int sparvar_decide_blocks(const void* q, const void* k, int B, int H
                           int32_t* kv_idx, float* mass, int32_t* dev_status, void* stream);
 
 /*
+ * Dense attention at the CS4A decision scale with the decision fused in: one
+ * launch computes O and the row LSE of attention over the whole key prefix
+ * (every KV block, no mask) and, from the same score tiles, the pooled mass and
+ * the selected lists of sparvar_decide_blocks ("Methodology in Plain English",
+ * CS4A paragraph: full attention at the decision scale, its weights summed per
+ * block, the top blocks kept).  Each 128-row query tile walks the prefix twice:
+ * a first sweep of score MMAs forms each row's log-sum-exp, the second computes
+ * P = exp(s - lse) (normalised), O += P V and the per-block sums of P.
+ *
+ * q, o [B][H][Lq][D], k, v [B][H][Lkv][D]: device bf16 with element strides for
+ *   (b, h, row) in host arrays *_strides[3]; last dim contiguous; base addresses
+ *   and row strides 16-byte aligned; D in {64, 128}.  ceil(Lkv / 128) <= 128.
+ * lse        device fp32 [B][H][Lq] (natural log) or NULL.
+ * softmax_scale, mass_threshold, topk_ratio: as for sparvar_decide_blocks
+ *   (blocks of 128 x 128).
+ * kv_cnt     device int32 [B][H][nqb]; kv_idx device int32 [B][H][nqb][nkb]: out.
+ * mass       device fp32 [B][H][nqb][nkb] or NULL: out.
+ * dev_status device int32 or NULL (SPARVAR_DEV_TIMEOUT on a wait that gave up).
+ * Errors: SPARVAR_ERR_UNSUPPORTED for D or the key count, SPARVAR_ERR_INVALID_ARG
+ * for bad pointers, strides or sizes; nothing is enqueued on an error return.
+ */
+SPARVAR_API int sparvar_decision_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                          float* lse, int B, int H, int Lq, int Lkv, int D,
+                                          const int64_t* q_strides, const int64_t* k_strides,
+                                          const int64_t* v_strides, const int64_t* o_strides,
+                                          float softmax_scale, float mass_threshold,
+                                          float topk_ratio, int32_t* kv_cnt, int32_t* kv_idx,
+                                          float* mass, int32_t* dev_status, void* stream);
+
+/*
  * CS4A cross-scale index mapping ("Methodology in Plain English", CS4A
  * paragraph: kept positions are rescaled to a later, larger scale, optionally
  * adding the sink region).

@@ -425,6 +425,58 @@ def test_decide_blocks_topk_ratio(ratio, D):
                     assert np.array_equal(idx[b, h, qb, :kk], oidx[qb, :kk])
 
 
+@pytest.mark.parametrize("scale_idx,D,B,H,tau,ratio", [
+    (9, 128, 1, 4, 0.95, 0.0),   # the 32x32 decision scale over its 2521-key prefix
+    (9, 128, 2, 2, 0.0, 0.2),    # the same with the Top-K rule
+    (8, 64, 1, 3, 0.9, 0.0),     # 24x24: 576 queries (a ragged last query tile), 1497 keys
+    (10, 128, 1, 2, 0.5, 0.0),   # 40x40: 1600 queries, 4121 keys (33 KV blocks)
+])
+def test_decision_attn_fwd_fused(scale_idx, D, B, H, tau, ratio):
+    """Dense attention with the CS4A decision fused in (one launch): O and LSE against
+    the fp64 oracle's dense attention, the pooled mass against the oracle's, every
+    list a valid selection of the kernel's own masses and bit-exact beyond the
+    margin, and the same masses as the stand-alone decision kernel."""
+    d = inputs.make_qkv(20 + scale_idx, B, H, INF, D, 5)
+    off = d["offsets"]
+    s = scale_idx
+    q_bits = d["q"][:, :, off[s]:off[s + 1]]
+    k_bits, v_bits = d["k"][:, :, :off[s + 1]], d["v"][:, :, :off[s + 1]]
+    st = _status()
+    o, lse, cnt, idx, mass = ops.sparvar_decision_attn_fwd(_dev(q_bits), _dev(k_bits), _dev(v_bits),
+                                                           tau, topk_ratio=ratio, return_mass=True,
+                                                           dev_status=st)
+    c2, i2, m2 = ops.sparvar_decide_blocks(_dev(q_bits), _dev(k_bits), tau, lse=lse,
+                                           topk_ratio=ratio, return_mass=True)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    cnt, idx, mass, m2 = cnt.cpu().numpy(), idx.cpu().numpy(), mass.cpu().numpy(), m2.cpu().numpy()
+    assert np.abs(mass - m2).max() < 2e-5
+    Lq, Lkv = q_bits.shape[2], k_bits.shape[2]
+    nqb, nkb = -(-Lq // 128), -(-Lkv // 128)
+    for b in range(B):
+        for h in range(H):
+            qf, kf, vf = q_bits_f(q_bits, b, h), q_bits_f(k_bits, b, h), q_bits_f(v_bits, b, h)
+            O, L = orc.masked_attention(qf, kf, vf, np.ones((nqb, nkb), bool), 128, 128)
+            err = np.abs(o[b, h] - O)
+            assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (b, h, err.max(), err.mean())
+            assert np.abs(lse[b, h] - L).max() < 1e-3
+            if ratio > 0:
+                oc, oi, _, M, margin = orc.decide_blocks(qf, kf, 128, 128, None, topk_ratio=ratio)
+            else:
+                oc, oi, _, M, margin = orc.decide_blocks(qf, kf, 128, 128, tau)
+            assert np.abs(mass[b, h] - M).max() < 2e-5
+            for qb in range(nqb):
+                if ratio > 0:
+                    err_s = topk_selection_error(cnt[b, h, qb], idx[b, h, qb], mass[b, h, qb],
+                                                 orc.topk_count(ratio, nkb))
+                else:
+                    err_s = mass_selection_error(cnt[b, h, qb], idx[b, h, qb], mass[b, h, qb], tau)
+                assert err_s == "", (b, h, qb, err_s)
+                if margin[qb] > 1e-4:
+                    assert cnt[b, h, qb] == oc[qb] and np.array_equal(idx[b, h, qb], oi[qb])
+
+
 @pytest.mark.parametrize("tau", [0.5, 0.99, 2.0])
 def test_decide_blocks_thresholds_d64(tau):
     d = inputs.make_qkv(2, 1, 2, INF, 64, 5)
