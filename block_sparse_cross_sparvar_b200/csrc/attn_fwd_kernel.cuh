@@ -28,10 +28,11 @@
 // softmax rescale O_s in place.  The two streams' groups alternate on the
 // tensor core while each stream's softmax works on its next block.
 //
-// Softmax per block: the row max of the 128 scores (columns 0-95 stay in
-// registers), a lazily raised reference (O is rescaled only when the block max
-// exceeds the reference by more than 2^8), then P = 2^(s * scale - m) in packed
-// f32x2 arithmetic with columns 96-127 re-read meanwhile.  Keys past the
+// Softmax per block: the 128 scores of a row stay in registers; P = 2^(s * scale
+// - m) in packed f32x2 arithmetic against a lazily raised reference m, with the
+// block's row max formed alongside; only when the block max exceeds the
+// reference by more than 2^8 (rare after a tile's first block) are O and the row
+// sum rescaled and the block redone.  A tile's first block takes its max first.  Keys past the
 // prefix, keys of fine blocks the tile mask drops and, with the token mask, keys
 // outside the CSLA rule are set to -inf first (one 128-bit keep mask per row).
 // Epilogue per tile: wait until the stream's last PV of the pair is complete and
@@ -44,6 +45,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "select.cuh"
 #include "tmem_io.cuh"
@@ -55,6 +58,11 @@ constexpr int kTile = 128;
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kIssuerWarp = 8;
 constexpr int kProducerWarp = 9;
+// flags of a ring item (item_meta_sh): kItemV a V block (else K); per stream st,
+// shifted by st: kItemUse the stream's MMA reads it, kItemFirst its first score /
+// PV MMA of the tile, kItemLast its last one; kItemEnd: no more items
+constexpr uint32_t kItemV = 1u << 8, kItemEnd = 1u << 9;
+constexpr uint32_t kItemUse = 1u << 0, kItemFirst = 1u << 2, kItemLast = 1u << 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.0f;          // log2 units
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
@@ -65,9 +73,9 @@ constexpr int kOutBoxRows = 32;               // rows of one output TMA store (o
 constexpr int kMaxDecBlocks = 128;            // KV blocks of a decision-scale prefix
 // Register budgets: the kernel is launched with kLaunchRegs per thread (the host
 // checks the compiled count); warps 8-11 (issuers, producers) give registers back
-// and the two softmax warpgroups take them: 2 * 128 * 208 + 128 * 88 = 384 * 168.
+// and the two softmax warpgroups take them: 2 * 128 * 200 + 128 * 104 = 384 * 168.
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 208, kControlRegs = 88;
+constexpr uint32_t kSoftmaxRegs = 200, kControlRegs = 104;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs,
               "register budgets exceed the launch allocation");
 
@@ -137,10 +145,10 @@ struct __align__(8) StreamBars {
 // the entries of the pair queue.
 struct __align__(8) SharedBars {
   uint64_t full[kMaxSlots];    // ring slot loaded                                 [u]
-  uint64_t empty[kMaxSlots];   // every MMA reading the slot is complete           [u]
+  uint64_t empty[kMaxSlots];   // the MMAs reading the slot are complete          [u]
   uint64_t tq_full[kTq];       // pair queue entry written                         [e]
-  uint64_t tq_empty[kTq];      // entry read by the issuer and the 256 softmax threads
-  uint64_t drain;
+  uint64_t tq_empty[kTq];      // entry read by the 256 softmax threads
+  uint64_t drain;              // the issuer's MMAs are complete
 };
 
 template <int D>
@@ -339,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ StreamBars bars_sh[2];
   __shared__ SharedBars sb;
   __shared__ int tq_pair_sh[kTq];
+  __shared__ uint32_t item_meta_sh[kMaxSlots];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float mass_sh[DEC ? 2 : 1][DEC ? kMaxDecBlocks : 1];     // decision: block sums
@@ -377,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kTq; ++i) {
       mbar_init(&sb.tq_full[i], 1);
-      mbar_init(&sb.tq_empty[i], 1 + 256);
+      mbar_init(&sb.tq_empty[i], 256);
     }
     mbar_init(&sb.drain, 1);
     fence_barrier_init();
@@ -405,18 +414,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ producer
     if (lane == 0) {
       int e = 0;                  // pair queue entries written
-      int items = 0;              // ring loads issued
+      int items = 0;              // ring items issued
       int kq[2] = {0, 0};         // Q loads issued per stream (one per non-empty tile)
       int pos = 0;                // pairs claimed
       bool ok = true;
-      auto load = [&](const CUtensorMap* tm, int kb, const PairCoord& pc) {
+      // the next ring slot, once the MMAs that read its previous item are complete
+      auto acquire_slot = [&]() -> int {
         const int i = items % NS;
         if (!mbar_wait(&sb.empty[i], ((items / NS) & 1) ^ 1, abort_flag, dev_status, 0x2,
                        kWaitNs)) {
           ok = false;
-          return;
+          return -1;
         }
+        return i;
+      };
+      // one K or V block into the next slot, with the item's flags for the issuers
+      auto load = [&](const CUtensorMap* tm, int kb, const PairCoord& pc, uint32_t meta) {
+        const int i = acquire_slot();
+        if (i < 0) return;
         kb = kb < 0 ? -1 : (kb > pc.nkb ? pc.nkb : kb);  // out of range: zero-filled, masked
+        item_meta_sh[i] = meta;
         mbar_arrive_expect_tx(&sb.full[i], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
@@ -440,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kq[st];
       };
       while (ok) {
-        // claim the CTA's next pair and publish it to the issuer and the softmax warps
+        // claim the CTA's next pair and publish it to the softmax warps
         const int64_t P64 = blockIdx.x + static_cast<int64_t>(pos++) * gridDim.x;
         const int P = P64 < total ? static_cast<int>(P64) : -1;
         const int q = e % kTq;
@@ -452,36 +469,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++e;
         if (P < 0) break;
         const PairCoord pc = pair_coord<MULTI>(P, args);
+        {
+          // the next pair's Q tiles into L2 now, so that their loads after this pair's
+          // last score MMAs are short
+          const int64_t Pn = P64 + gridDim.x;
+          if (Pn < total) {
+            const PairCoord pn = pair_coord<MULTI>(static_cast<int>(Pn), args);
+            for (int st = 0; st < 2; ++st) {
+              if (2 * pn.pp + st >= pn.nqb) continue;
+#pragma unroll
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_prefetch_4d(&tm_q, c * 64, pn.row0 + (2 * pn.pp + st) * kTile, pn.h, pn.b);
+            }
+          }
+        }
         Merge<DEC> m{};
         m.n0 = stream_list<DEC>(pc, 0, args, true, &m.l0);
         m.n1 = stream_list<DEC>(pc, 1, args, true, &m.l1);
         if (m.n0 + m.n1 == 0) continue;
+        const int n[2] = {m.n0, m.n1};
+        const int npv[2] = {DEC ? m.n0 / 2 : m.n0, DEC ? m.n1 / 2 : m.n1};
+        int ns[2] = {0, 0}, nv[2] = {0, 0};  // score and PV items per stream so far
         if (m.n0 > 0) load_q(0, pc);
         if (ok && m.n1 > 0) load_q(1, pc);
+        // flags of the K item of the current entry and of the V item
+        auto k_meta = [&]() {
+          uint32_t f = 0;
+          const bool in[2] = {m.in0, m.in1};
+          for (int st = 0; st < 2; ++st) {
+            if (!in[st]) continue;
+            f |= kItemUse << st;
+            if (ns[st] == 0) f |= kItemFirst << st;
+            if (++ns[st] == n[st]) f |= kItemLast << st;
+          }
+          return f;
+        };
         // ring order: K of the first entry, then per entry: V (if the entry has PV
         // MMAs) and the K of the next entry
         m.next();
-        if (ok) load(&tm_k, m.kb, pc);
+        if (ok) load(&tm_k, m.kb, pc, k_meta());
         while (ok) {
           const int kb = m.kb;
           const bool pv = m.pv;
+          const bool in[2] = {m.in0, m.in1};
           const bool more = m.next();
-          if (pv) load(&tm_v, kb, pc);
+          if (pv) {
+            uint32_t f = kItemV;
+            for (int st = 0; st < 2; ++st) {
+              if (!in[st]) continue;
+              f |= kItemUse << st;
+              if (nv[st] == 0) f |= kItemFirst << st;
+              if (++nv[st] == npv[st]) f |= kItemLast << st;
+            }
+            load(&tm_v, kb, pc, f);
+          }
           if (!more || !ok) break;
-          load(&tm_k, m.kb, pc);
+          load(&tm_k, m.kb, pc, k_meta());
+        }
+      }
+      // the end of the item stream for the issuers
+      if (ok) {
+        const int i = acquire_slot();
+        if (i >= 0) {
+          item_meta_sh[i] = kItemEnd;
+          mbar_arrive(&sb.full[i]);
+          ++items;
         }
       }
       // drain: every issued TMA write lands before the CTA exits
       for (int st = 0; st < 2; ++st)
         if (kq[st] > 0) mbar_drain(&bars_sh[st].q_full, (kq[st] - 1) & 1, kDrainNs);
       for (int i = 0; i < NS; ++i) {
-        const int issued = items > i ? (items - 1 - i) / NS + 1 : 0;  // loads into slot i
+        const int issued = items > i ? (items - 1 - i) / NS + 1 : 0;  // items in slot i
         if (issued) mbar_drain(&sb.full[i], (issued - 1) & 1, kDrainNs);
       }
     }
     __syncwarp();
    } else if (warp == kIssuerWarp) {
     // ================================================================ MMA issue
+    // The issuer follows the ring items in order, taking a V item together with the
+    // K item after it.  For each stream that uses them it issues the group [PV of
+    // the stream's block on V, S of its next block on K]; the streams' groups go to
+    // the tensor core one after the other, whichever stream's P is ready first.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, D, 1);
@@ -489,109 +558,103 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = smem_desc_sw128(sQ(0), 16, 1024);
       const uint64_t dk = smem_desc_sw128(sSlot(0), 16, 1024);
       const uint64_t dv = smem_desc_sw128(sSlot(0), L::kChunkBytes, 1024);
-      int e = 0, items = 0;
-      int J[2] = {0, 0};  // blocks per stream (s_full / p_full phases)
-      int k[2] = {0, 0};  // non-empty tiles per stream (q_full / q_free / o_done phases)
-      bool ok = true;
-      auto wait_item = [&]() -> int {
+      int items = 0;
+      // per stream: p_full waits (one per block), tiles (q_full / q_free phases), and
+      // whether a block's P has not been waited for yet (no PV since its S)
+      int J0 = 0, J1 = 0, k0 = 0, k1 = 0;
+      bool pp0 = false, pp1 = false;
+      bool ok = true, end = false;
+      auto next_item = [&](uint32_t& meta) -> int {
         const int i = items % NS;
         ok = ok && mbar_wait(&sb.full[i], (items / NS) & 1, abort_flag, dev_status, 0x2, kWaitNs);
         ++items;
+        meta = ok ? item_meta_sh[i] : kItemEnd;
         return i;
       };
-      // S_st = Q_st K^T with K in ring slot i, into S_st
-      auto issue_s = [&](int st, int i) {
-        const uint64_t dqs = dq + static_cast<uint64_t>(st * kBufStep);
-        const uint64_t dks = dk + static_cast<uint64_t>(i * kBufStep);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + 256u * st, dqs + off, dks + off, idesc_s, kk > 0 ? 1u : 0u);
+      // stream st's group on V slot iv (flags vm) and K slot ik (flags km), if it is
+      // ready; returns whether it was issued
+      auto group = [&](auto stc, uint32_t vm, uint32_t km, int iv, int ik, int& J, int& k,
+                       bool& pp) -> bool {
+        constexpr int st = decltype(stc)::value;
+        StreamBars& bs = bars_sh[st];
+        const bool use_v = (vm >> st) & kItemUse, use_k = (km >> st) & kItemUse;
+        const bool need_p = use_v || (use_k && pp);
+        if (need_p && !mbar_try_wait(&bs.p_full, J & 1)) return false;
+        if (use_k && ((km >> st) & kItemFirst) && !mbar_try_wait(&bs.q_full, k & 1)) return false;
+        if (need_p) {
+          ++J;
+          pp = false;
         }
+        tc_fence_after();
+        const uint32_t s_col = tmem + 256u * st;
+        if (use_v) {
+          const uint64_t dvs = dv + static_cast<uint64_t>(iv * kBufStep);
+          const uint32_t acc0 = ((vm >> st) & kItemFirst) ? 0u : 1u;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(s_col + 128, s_col + kk * 8, dvs + static_cast<uint64_t>(kk * (2048 >> 4)),
+                   idesc_pv, kk > 0 ? 1u : acc0);
+          if ((vm >> st) & kItemLast) mma_commit(&bs.o_done);
+        }
+        if (use_k) {
+          const uint64_t dqs = dq + static_cast<uint64_t>(st * kBufStep);
+          const uint64_t dks = dk + static_cast<uint64_t>(ik * kBufStep);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+            mma_ss(s_col, dqs + off, dks + off, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          if ((km >> st) & kItemLast) {
+            mma_commit(&bs.q_free);
+            ++k;
+          }
+          mma_commit(&bs.s_full);
+          pp = true;
+        }
+        return true;
       };
-      while (ok) {
-        const int q = e % kTq;
-        if (!mbar_wait(&sb.tq_full[q], (e / kTq) & 1, abort_flag, dev_status, 0x2, kWaitNs)) break;
-        const int P = tq_pair_sh[q];
-        mbar_arrive(&sb.tq_empty[q]);
-        ++e;
-        if (P < 0) break;
-        const PairCoord pc = pair_coord<MULTI>(P, args);
-        Merge<DEC> m{};
-        m.n0 = stream_list<DEC>(pc, 0, args, false, &m.l0);
-        m.n1 = stream_list<DEC>(pc, 1, args, false, &m.l1);
-        if (m.n0 + m.n1 == 0) continue;
-        const int n[2] = {m.n0, m.n1};
-        const int npv[2] = {DEC ? m.n0 / 2 : m.n0, DEC ? m.n1 / 2 : m.n1};
-        int ns[2] = {0, 0}, nv[2] = {0, 0};  // score and PV MMAs issued per stream in this pair
-        for (int st = 0; st < 2 && ok; ++st)
-          if (n[st] > 0)
-            ok = mbar_wait(&bars_sh[st].q_full, k[st] & 1, abort_flag, dev_status, 0x2, kWaitNs);
-        // the score MMAs of the first entry
-        m.next();
-        {
-          const int ik = wait_item();
-          if (!ok) break;
-          tc_fence_after();
-          const bool in[2] = {m.in0, m.in1};
-          for (int st = 0; st < 2; ++st) {
-            if (!in[st]) continue;
-            issue_s(st, ik);
-            if (++ns[st] == n[st]) mma_commit(&bars_sh[st].q_free);
-            mma_commit(&bars_sh[st].s_full);
+      while (ok && !end) {
+        uint32_t m1, m2 = 0;
+        const int i1 = next_item(m1);
+        if (m1 & kItemEnd) break;
+        int iv = -1, ik = i1;
+        uint32_t vm = 0, km = m1;
+        if (m1 & kItemV) {
+          iv = i1;
+          vm = m1;
+          ik = next_item(m2);
+          km = m2;
+          if (m2 & kItemEnd) {
+            end = true;
+            ik = -1;
+            km = 0;
           }
-          mma_commit(&sb.empty[ik]);
         }
-        while (ok) {
-          const bool in[2] = {m.in0, m.in1};
-          const bool pv = m.pv;
-          const bool more = m.next();
-          const bool in_next[2] = {more && m.in0, more && m.in1};
-          const int iv = pv ? wait_item() : -1;
-          int ik = -1;
-          if (!ok) break;
-          for (int st = 0; st < 2 && ok; ++st) {
-            StreamBars& bs = bars_sh[st];
-            if (in[st]) {
-              // P of the stream's block (or, in the first decision sweep, S read) handed over
-              ok = mbar_wait(&bs.p_full, J[st] & 1, abort_flag, dev_status, 0x2, kWaitNs);
-              ++J[st];
-              if (!ok) break;
-              if (pv) {
-                tc_fence_after();
-                const uint64_t dvs = dv + static_cast<uint64_t>(iv * kBufStep);
-                const uint32_t o_col = tmem + 256u * st + 128;
-                const uint32_t p_col = tmem + 256u * st;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                  mma_ts(o_col, p_col + kk * 8, dvs + static_cast<uint64_t>(kk * (2048 >> 4)),
-                         idesc_pv, (nv[st] > 0 || kk > 0) ? 1u : 0u);
-                if (++nv[st] == npv[st]) mma_commit(&bs.o_done);
-              }
+        if (!ok) break;
+        // each stream's group, in the order the streams become ready
+        bool todo0 = (vm | km) & kItemUse, todo1 = ((vm | km) >> 1) & kItemUse;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t spin = 0; todo0 || todo1; ++spin) {
+          if (todo0 && group(std::integral_constant<int, 0>{}, vm, km, iv, ik, J0, k0, pp0))
+            todo0 = false;
+          if (todo1 && group(std::integral_constant<int, 1>{}, vm, km, iv, ik, J1, k1, pp1))
+            todo1 = false;
+          if ((spin & 15u) == 15u && (todo0 || todo1)) {
+            if (*abort_flag) {
+              ok = false;
+              break;
             }
-            if (in_next[st]) {
-              if (ik < 0) {
-                ik = wait_item();
-                if (!ok) break;
-              }
-              tc_fence_after();
-              issue_s(st, ik);
-              if (++ns[st] == n[st]) mma_commit(&bs.q_free);
-              mma_commit(&bs.s_full);
+            if (global_timer_ns() - t0 > kWaitNs) {
+              *abort_flag = 1;
+              if (dev_status) atomicOr(dev_status, 0x2);
+              ok = false;
+              break;
             }
           }
-          if (!ok) break;
-          if (iv >= 0) mma_commit(&sb.empty[iv]);
-          if (more && ik < 0) {
-            // an entry is always run by some stream, so its K has a reader
-            ik = wait_item();
-            if (!ok) break;
-          }
-          if (ik >= 0) mma_commit(&sb.empty[ik]);
-          if (!more) break;
         }
-        for (int st = 0; st < 2; ++st)
-          if (n[st] > 0) ++k[st];
+        if (!ok) break;
+        if (iv >= 0) mma_commit(&sb.empty[iv]);
+        if (ik >= 0) mma_commit(&sb.empty[ik]);
       }
       mma_commit(&sb.drain);
       mbar_drain(&sb.drain, 0, kDrainNs);
@@ -690,17 +753,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool masked = __any_sync(0xffffffffu, (km[0] & km[1] & km[2] & km[3]) != ~0u);
-        // pass 1: the block's row max.  Columns 0-95 stay in registers for pass 2.
-        float bm;
-        uint32_t s0[32], s1[32], s2[32];
-        {
-          uint32_t sr[kTile];
-          tmem_ld128_wait(s_addr, sr);
-          if (masked) {
+        // the block's 128 scores of this row, in registers for the whole block
+        uint32_t sr[kTile];
+        tmem_ld128_wait(s_addr, sr);
+        if (masked) {
 #pragma unroll
-            for (int c = 0; c < kTile; ++c)
-              if (!((km[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
-          }
+          for (int c = 0; c < kTile; ++c)
+            if (!((km[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
+        }
+        auto row_max = [&]() {
           float mx0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[4]));
           float mx1 = fmaxf(__uint_as_float(sr[1]), __uint_as_float(sr[5]));
           float mx2 = fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[6]));
@@ -712,39 +773,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx2 = max3(mx2, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 6]));
             mx3 = max3(mx3, __uint_as_float(sr[c + 3]), __uint_as_float(sr[c + 7]));
           }
-          bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * csc;
-          if (sweep_a) {
-            // the row's running log-sum-exp: reference max(m, bm), sum rescaled exactly
-            const float m_new = fmaxf(m_run, bm);
-            const float nm = m_new == -INFINITY ? 0.f : -m_new;
-            const uint64_t sc2 = f2_pack(csc, csc), nm2 = f2_pack(nm, nm);
-            uint64_t a0 = 0, a1 = 0;
-#pragma unroll
-            for (int c = 0; c < kTile; c += 4) {
-              float e0, e1, e2, e3;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2,
-                               nm2),
-                        e0, e1);
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sc2,
-                               nm2),
-                        e2, e3);
-              a0 = f2_add(a0, f2_pack(ex2_approx(e0), ex2_approx(e1)));
-              a1 = f2_add(a1, f2_pack(ex2_approx(e2), ex2_approx(e3)));
-            }
-            float x0, x1;
-            f2_unpack(f2_add(a0, a1), x0, x1);
-            l_run = (m_run == -INFINITY ? 0.f : l_run * ex2_approx(m_run - m_new)) + x0 + x1;
-            m_run = m_new;
-          }
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            s0[c] = sr[c];
-            s1[c] = sr[32 + c];
-            s2[c] = sr[64 + c];
-          }
-        }
+          return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * csc;
+        };
         if (sweep_a) {
-          // S has been read: the next score MMA may overwrite it
+          // decision, first sweep: the row's running log-sum-exp, reference max(m, bm),
+          // the sum rescaled exactly; S has been read, so the next score MMA may
+          // overwrite it
+          const float bm = row_max();
+          const float m_new = fmaxf(m_run, bm);
+          const float nm = m_new == -INFINITY ? 0.f : -m_new;
+          const uint64_t sc2 = f2_pack(csc, csc), nm2 = f2_pack(nm, nm);
+          uint64_t a0 = 0, a1 = 0;
+#pragma unroll
+          for (int c = 0; c < kTile; c += 4) {
+            float e0, e1, e2, e3;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2),
+                      e0, e1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sc2,
+                             nm2),
+                      e2, e3);
+            a0 = f2_add(a0, f2_pack(ex2_approx(e0), ex2_approx(e1)));
+            a1 = f2_add(a1, f2_pack(ex2_approx(e2), ex2_approx(e3)));
+          }
+          float x0, x1;
+          f2_unpack(f2_add(a0, a1), x0, x1);
+          l_run = (m_run == -INFINITY ? 0.f : l_run * ex2_approx(m_run - m_new)) + x0 + x1;
+          m_run = m_new;
           if (j + 1 == n / 2) {
             // end of the sweep: the row's log-sum-exp is the fixed reference of the
             // second sweep, whose P is then already normalised
@@ -755,63 +809,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bs.p_full);
           continue;
         }
-        // the reference: set by the first finite block max, raised when a block max
-        // exceeds it by more than 2^8 (O and the row sum are rescaled then)
-        const bool raise =
-            !DEC && (m_run == -INFINITY ? (bm != -INFINITY) : (bm > m_run + kLazyRescale));
-        const bool o_live = raise && m_run != -INFINITY;
-        if (__any_sync(0xffffffffu, o_live)) {
-          // S(j) complete implies PV(j - 1) complete: O is quiescent
-          const float alpha = o_live ? ex2_approx(m_run - bm) : 1.f;
-          l_run *= alpha;
+        // O and the row sum move to a new reference m_new (per lane; O is quiescent:
+        // S(j) complete implies PV(j - 1) complete)
+        auto raise_to = [&](bool raise, float m_new) {
+          const bool o_live = raise && m_run != -INFINITY;
+          if (__any_sync(0xffffffffu, o_live)) {
+            const float alpha = o_live ? ex2_approx(m_run - m_new) : 1.f;
+            l_run *= alpha;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t orr[16];
+              tmem_ld16_wait(o_addr + cc * 16, orr);
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t orr[32];
-            tmem_ld32_wait(o_addr + cc * 32, orr);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-            tmem_st32(o_addr + cc * 32, orr);
-          }
-        }
-        if (raise) m_run = bm;
-        const float neg = (m_run == -INFINITY) ? 0.f : -m_run;
-        // pass 2: P = 2^(s * scale - m) in packed pairs.  Columns 96-127 are re-read
-        // while the columns held in registers are worked on; P chunk cc (packed bf16)
-        // overwrites TMEM columns [16cc, 16cc + 16), already read.
-        const uint64_t sc2 = f2_pack(csc, csc), neg2 = f2_pack(neg, neg);
-        uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
-        auto p_chunk = [&](const uint32_t(&cur)[32], int cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float e0, e1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
-                             sc2, neg2),
-                      e0, e1);
-            const float p0 = ex2_approx(e0);
-            const float p1 = ex2_approx(e1);
-            if (c & 1) {
-              acc1 = f2_add(acc1, f2_pack(p0, p1));
-            } else {
-              acc0 = f2_add(acc0, f2_pack(p0, p1));
+              for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+              tmem_st16(o_addr + cc * 16, orr);
             }
-            pk[c] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(s_addr + cc * 16, pk);
+          if (raise) m_run = m_new;
         };
-        {
-          uint32_t s3[32];
-          tmem_ld32_async(s_addr + 96, s3, __float_as_uint(neg));
-          p_chunk(s0, 0);
-          p_chunk(s1, 1);
-          p_chunk(s2, 2);
-          tmem_wait_ld_tied(s3);
-          if (masked) {
+        // P = 2^(s * scale - m) in packed pairs, written over TMEM columns [8cc, 8cc + 8)
+        // of the scores (already in registers) as packed bf16; with TRACK the raw row max
+        // is formed alongside (it fills issue slots the exponentials leave free)
+        const uint64_t sc2 = f2_pack(csc, csc);
+        uint64_t acc0 = 0, acc1 = 0;  // (0.f, 0.f)
+        auto exp_pass = [&](auto track) {
+          const float neg = (m_run == -INFINITY) ? 0.f : -m_run;
+          const uint64_t neg2 = f2_pack(neg, neg);
+          float t0 = -INFINITY, t1 = -INFINITY;
+          acc0 = acc1 = 0;
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (!((km[3] >> c) & 1u)) s3[c] = __float_as_uint(-INFINITY);
+          for (int cc = 0; cc < kTile / 16; ++cc) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float x0 = __uint_as_float(sr[cc * 16 + 2 * c]);
+              const float x1 = __uint_as_float(sr[cc * 16 + 2 * c + 1]);
+              if constexpr (decltype(track)::value) {
+                if (c & 1) {
+                  t1 = max3(t1, x0, x1);
+                } else {
+                  t0 = max3(t0, x0, x1);
+                }
+              }
+              float e0, e1;
+              f2_unpack(f2_fma(f2_pack(x0, x1), sc2, neg2), e0, e1);
+              const float p0 = ex2_approx(e0);
+              const float p1 = ex2_approx(e1);
+              if (c & 1) {
+                acc1 = f2_add(acc1, f2_pack(p0, p1));
+              } else {
+                acc0 = f2_add(acc0, f2_pack(p0, p1));
+              }
+              pk[c] = pack_bf16x2(p0, p1);
+            }
+            tmem_st8(s_addr + cc * 8, pk);
           }
-          p_chunk(s3, 3);
+          return fmaxf(t0, t1) * csc;
+        };
+        if (DEC) {
+          // decision, second sweep: the fixed reference is the row's log-sum-exp
+          exp_pass(std::false_type{});
+        } else if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
+          // a row without a reference yet (a tile's first block): the block max first
+          const float bm = row_max();
+          raise_to(m_run == -INFINITY ? (bm != -INFINITY) : (bm > m_run + kLazyRescale), bm);
+          exp_pass(std::false_type{});
+        } else {
+          // against the current reference, the block max formed alongside; in the rare
+          // case that it exceeds the reference by more than 2^8 the reference is raised
+          // and the block redone
+          const float bm = exp_pass(std::true_type{});
+          const bool raise = bm > m_run + kLazyRescale;
+          if (__any_sync(0xffffffffu, raise)) {
+            tmem_wait_st();
+            raise_to(raise, bm);
+            exp_pass(std::false_type{});
+          }
         }
         {
           float a0, a1;

@@ -4,10 +4,10 @@ A small discrete model of the persistent attn_fwd_kernel.cuh: one CTA claiming
 pairs of query tiles (two streams, one tile each) that share one K/V stream:
 the TMA producer, the MMA issuer and four softmax warps per stream, with the
 tensor core and the TMA engine, connected by mbarriers with phase counters.
-Random interleavings (TMA loads landing in any order, random "raise the
-reference max" decisions) are explored for many pair sequences (empty lists,
-missing second tiles, one-block tiles, disjoint and overlapping lists, lists out
-of order) and ring sizes, checking
+Random interleavings (either stream's MMA group first when both are ready, TMA
+loads landing in any order, random "raise the reference max" decisions) are explored
+for many pair sequences (empty lists, missing second tiles, one-block tiles,
+disjoint and overlapping lists, lists out of order) and ring sizes, checking
 
 * that no schedule deadlocks;
 * that every parity wait only observes its own phase or the next one (a barrier
@@ -20,20 +20,24 @@ of order) and ring sizes, checking
   stream's MMAs see its own list in its own order.
 
 The model follows the kernel step for step.  The producer claims a pair,
-publishes it in the pair queue, loads each stream's Q once that stream's
-previous tile's last score MMA is complete (q_free), and loads ring items in the
-order K of the first merged entry, then per entry: V and the K of the next
-entry, each into slot (item mod NS) once the MMAs that read the slot's previous
-item are complete.  The issuer waits for the streams' Q, issues the score MMAs
-of the first entry, then per entry, for stream 0 then 1: wait P (if the stream
-keeps the entry), PV [o_done after the stream's last PV of the pair], the
-stream's next score MMA if it keeps the next entry [q_free after its last one;
-s_full]; then it frees the entry's two slots.  Each softmax warp waits
-s_full(J), may rescale O, writes P and arrives on p_full; after a tile's last
-block it waits o_done and reads O, before it can arrive on p_full for its next
-tile's first block.  Known-bad variants (the epilogue's O read deferred past
-the next tile's first block, no q_free wait, no wait for the previous use of a
-ring slot) are checked to be caught, so the checker is not vacuous.
+publishes it in the pair queue for the softmax warps, loads each stream's Q once
+that stream's previous tile's last score MMA is complete (q_free), and loads
+ring items in the order K of the first merged entry, then per entry: V and the
+K of the next entry, each into slot (item mod NS) once the MMAs that read the
+slot's previous item are complete, with flags saying which streams use the
+item and whether it is a stream's first or last score / PV item of its tile;
+a final item marks the end.  The issuer takes a V item together with the K item
+after it and, for each stream that uses them, as soon as that stream's P (and,
+for a tile's first score MMA, its Q) is ready, issues the stream's group: PV on
+V [o_done after the tile's last], S on K [q_free after the tile's last;
+s_full]; a K item alone (a pair's first) waits for the previous block's P when
+no PV did.  Then it releases both slots.  Each softmax
+warp waits s_full(J), may rescale O, writes P and arrives on p_full; after a
+tile's last block it waits o_done and reads O, before it can arrive on p_full
+for its next tile's first block.  Known-bad variants (the epilogue's O read
+deferred past the next tile's first block, no q_free wait, no wait for the
+previous use of a ring slot, releasing a slot before the MMA that reads it)
+are checked to be caught, so the checker is not vacuous.
 """
 import random
 
@@ -91,7 +95,7 @@ class Model:
             self.bars[("empty", i)] = Bar()
         for i in range(tq):
             self.bars[("tq_full", i)] = Bar()
-            self.bars[("tq_empty", i)] = Bar(1 + 2 * N_WARPS)
+            self.bars[("tq_empty", i)] = Bar(2 * N_WARPS)
         self.queue = {}
         self.q_buf = {0: None, 1: None}
         self.slot = {i: None for i in range(ns)}
@@ -100,6 +104,8 @@ class Model:
         self.pv_inflight = {0: 0, 1: 0}
         self.o_reads = {}
         self.seen = {0: [], 1: []}  # KV blocks each stream's score MMAs read, in order
+        self.meta = {}  # ring item number -> flags
+        self.item_kb = {}  # ring item number -> KV block
         self.tc = []  # the issuer's tensor-core queue (in order)
         self.tma = []
         self.roles = [self.producer(), self.issuer()]
@@ -107,6 +113,9 @@ class Model:
             for w in range(N_WARPS):
                 self.roles.append(self.softmax(s, w))
         self.cur = [next(r) for r in self.roles]
+
+    def slot_kb(self, item):
+        return self.item_kb[item]
 
     def lists(self, p):
         l0, l1 = self.pairs[p]
@@ -116,12 +125,17 @@ class Model:
     def producer(self):
         e, items, kq = 0, 0, [0, 0]
 
-        def load(kb):
+        def load(kb, meta):
             nonlocal items
             i = items % self.ns
             if items >= self.ns and "no_slot_wait" not in self.bad:
                 yield ("wait", ("empty", i), items // self.ns - 1)
-            yield ("tma", ("full", i), ("slot", i, (items, kb)))
+            self.meta[items] = meta
+            self.item_kb[items] = kb
+            if meta["kind"] == "end":
+                yield ("arrive", ("full", i))
+            else:
+                yield ("tma", ("full", i), ("slot", i, (items, kb)))
             items += 1
 
         for p in list(range(len(self.pairs))) + [None]:
@@ -143,77 +157,105 @@ class Model:
             ent = merge(*ls)
             if not ent:
                 continue
-            yield from load(ent[0][0])
-            for u, (kb, _, _) in enumerate(ent):
-                yield from load(kb)  # V
+            n = [len(ls[0]), len(ls[1])]
+            ns_, nv = [0, 0], [0, 0]
+
+            def flags(kind, ins, cnt, tot):
+                f = {"kind": kind, "use": [False, False], "first": [False, False],
+                     "last": [False, False]}
+                for s in (0, 1):
+                    if ins[s]:
+                        f["use"][s] = True
+                        f["first"][s] = cnt[s] == 0
+                        cnt[s] += 1
+                        f["last"][s] = cnt[s] == tot[s]
+                return f
+
+            yield from load(ent[0][0], flags("K", ent[0][1:], ns_, n))
+            for u, (kb, a0, a1) in enumerate(ent):
+                yield from load(kb, flags("V", (a0, a1), nv, n))
                 if u + 1 < len(ent):
-                    yield from load(ent[u + 1][0])  # K of the next entry
+                    yield from load(ent[u + 1][0], flags("K", ent[u + 1][1:], ns_, n))
+        yield from load(None, {"kind": "end"})
         yield ("end",)
 
     def issuer(self):
-        e, items = 0, 0
-        J, k = [0, 0], [0, 0]
+        """The single issuer: a V item together with the K item after it; each stream's
+        group [PV on V, S on K] as soon as that stream is ready, in either order."""
+        items = 0
+        J, k, kpv = [0, 0], [0, 0], [0, 0]
+        pp = [False, False]
 
-        def wait_item():
+        def next_item():
             nonlocal items
             i = items % self.ns
             yield ("wait", ("full", i), items // self.ns)
+            it = items
             items += 1
-            return i, items - 1
+            return i, it, self.meta[it]
 
-        while True:
-            q = e % self.tq
-            yield ("wait", ("tq_full", q), e // self.tq)
-            p = self.queue[e]
-            yield ("arrive", ("tq_empty", q))
-            e += 1
-            if p is None:
+        end = False
+        while not end:
+            i1, it1, m1 = yield from next_item()
+            if m1["kind"] == "end":
                 break
-            ls = self.lists(p)
-            ent = merge(*ls)
-            if not ent:
-                continue
-            n = [len(ls[0]), len(ls[1])]
-            ns_, nv = [0, 0], [0, 0]
-            for s in (0, 1):
-                if n[s]:
-                    yield ("wait", (s, "q_full"), k[s])
-            ik, it = yield from wait_item()
-            for s in (0, 1):
-                if ent[0][1 + s]:
-                    yield ("mma", ("S", s, J[s] + ns_[s], (s, k[s]), ik, it, ent[0][0]))
-                    ns_[s] += 1
-                    if ns_[s] == n[s]:
+            v = k_ = None
+            if m1["kind"] == "V":
+                v = (i1, it1, m1)
+                i2, it2, m2 = yield from next_item()
+                if m2["kind"] == "end":
+                    end = True
+                else:
+                    k_ = (i2, it2, m2)
+            else:
+                k_ = (i1, it1, m1)
+            todo = [s for s in (0, 1) if (v and v[2]["use"][s]) or (k_ and k_[2]["use"][s])]
+            while todo:
+                # the streams whose group can go now (P and Q ready); the model lets any
+                # ready stream go first
+                ready = []
+                for s in todo:
+                    use_v = v is not None and v[2]["use"][s]
+                    use_k = k_ is not None and k_[2]["use"][s]
+                    need = []
+                    if use_v or (use_k and pp[s]):
+                        need.append(((s, "p_full"), J[s]))
+                    if use_k and k_[2]["first"][s]:
+                        need.append(((s, "q_full"), k[s]))
+                    if all(self.ready(("wait", b, ph)) for b, ph in need):
+                        ready.append(s)
+                if not ready:
+                    yield ("poll",)
+                    continue
+                s = self.rng.choice(ready)
+                todo.remove(s)
+                use_v = v is not None and v[2]["use"][s]
+                use_k = k_ is not None and k_[2]["use"][s]
+                if use_v or (use_k and pp[s]):
+                    J[s] += 1
+                    pp[s] = False
+                if use_v:
+                    i, it, m = v
+                    yield ("mma", ("PV", s, J[s] - 1, (s, kpv[s]), i, it, m["first"][s],
+                                   self.slot_kb(it)))
+                    if m["last"][s]:
+                        yield ("commit", (s, "o_done"))
+                        kpv[s] += 1
+                if use_k:
+                    i, it, m = k_
+                    yield ("mma", ("S", s, J[s], (s, k[s]), i, it, self.slot_kb(it)))
+                    if m["last"][s]:
                         yield ("commit", (s, "q_free"))
+                        k[s] += 1
                     yield ("commit", (s, "s_full"))
-            yield ("commit", ("empty", ik))
-            for u, (kb, a0, a1) in enumerate(ent):
-                ins = (a0, a1)
-                nxt = ent[u + 1] if u + 1 < len(ent) else None
-                iv, itv = yield from wait_item()
-                ik = None
-                for s in (0, 1):
-                    if ins[s]:
-                        yield ("wait", (s, "p_full"), J[s])
-                        yield ("mma", ("PV", s, J[s], (s, k[s]), iv, itv, nv[s] == 0, kb))
-                        J[s] += 1
-                        nv[s] += 1
-                        if nv[s] == n[s]:
-                            yield ("commit", (s, "o_done"))
-                    if nxt is not None and nxt[1 + s]:
-                        if ik is None:
-                            ik, itk = yield from wait_item()
-                        yield ("mma", ("S", s, J[s], (s, k[s]), ik, itk, nxt[0]))
-                        ns_[s] += 1
-                        if ns_[s] == n[s]:
-                            yield ("commit", (s, "q_free"))
-                        yield ("commit", (s, "s_full"))
-                yield ("commit", ("empty", iv))
-                if ik is not None:
-                    yield ("commit", ("empty", ik))
-            for s in (0, 1):
-                if n[s]:
-                    k[s] += 1
+                    pp[s] = True
+            if v is not None:
+                if "early_release" in self.bad:
+                    yield ("arrive", ("empty", v[0]))
+                else:
+                    yield ("commit", ("empty", v[0]))
+            if k_ is not None:
+                yield ("commit", ("empty", k_[0]))
         yield ("commit", "drain")
         yield ("wait", "drain", 0)
         yield ("end",)
@@ -352,7 +394,7 @@ class Model:
                     self.tc.append(op)
                 elif op[0] == "arrive":
                     self.bars[op[1]].arrive()
-                elif op[0] != "wait":
+                elif op[0] not in ("wait", "poll"):
                     self.effect(op)
                 self.cur[i] = next(self.roles[i])
         raise AssertionError("model did not finish")
@@ -419,10 +461,16 @@ def test_late_epilogue_is_caught():
 def test_missing_q_free_wait_is_caught():
     """Without the q_free wait the next tile's Q can land while a score MMA of the
     current tile still reads the buffer."""
-    assert _caught("no_q_free", [([0, 1], [1, 2]), ([0], [0]), ([2, 3], [1])], 2) > 0
+    assert _caught("no_q_free", [([0, 1], [1, 2]), ([0], [0]), ([2, 3], [1])], 4) > 0
 
 
 def test_missing_slot_wait_is_caught():
     """Without waiting for the previous use of a ring slot a load can overwrite an
     operand before its MMA has run."""
     assert _caught("no_slot_wait", [([0, 1, 2, 3, 4], [2, 3, 4, 5, 6])], 2) > 0
+
+
+def test_release_before_the_mma_is_caught():
+    """An issuer that released a V slot with a plain arrival (instead of a commit that
+    fires when its PV has read the slot) would let the next load overwrite V early."""
+    assert _caught("early_release", [([0, 1, 2, 3, 4], [1, 2, 3, 4, 5])], 2) > 0
