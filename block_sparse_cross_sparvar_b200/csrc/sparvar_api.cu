@@ -15,6 +15,7 @@
 #include "../../include/sparvar.h"
 #include "attn_fwd_kernel.cuh"
 #include "decide_kernel.cuh"
+#include "decision_attn_kernel.cuh"
 #include "mask_kernels.cuh"
 #include "ocache_kernel.cuh"
 #include "wait_probe_kernel.cuh"
@@ -81,8 +82,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 4-D map over a [B][H][rows][D] bf16 tensor: box = 64 columns x box_rows rows
-// (128 for loads, one warp's 32 rows for the attention output), 128-byte swizzle,
-// zero fill outside the tensor.
+// (128, a query or key tile; 32, one warp's rows of the decision kernel's output),
+// 128-byte swizzle, zero fill outside the tensor.
 int make_tmap(CUtensorMap* m, const void* base, int D, int rows, int H, int B, int64_t sr,
               int64_t sh, int64_t sb, const char* name, int box_rows = 128) {
   auto enc = tensor_map_encoder();
@@ -141,12 +142,40 @@ int launch_decide_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const spa
   return SPARVAR_OK;
 }
 
-template <int D, bool TOK, bool MULTI, bool DEC = false>
+template <int D, bool TOK, bool MULTI>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const sparvar::fwd::OutMaps& to, const sparvar::fwd::Args& a,
                       cudaStream_t stream) {
-  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI, DEC>;
+  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  // persistent: one CTA per SM, each walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
+  const int64_t tiles = a.total_tiles;
+  const int64_t grid = tiles < sms ? tiles : sms;
+  // the kernel's per-CTA sequence counters (blocks, ring positions) are 32-bit
+  int64_t row_len = 0;
+  for (int i = 0; i < a.n_problems; ++i) row_len = std::max<int64_t>(row_len, a.prob[i].idx_row_len);
+  if (ceil_div(tiles, grid) * (3 * row_len + 1) >= (int64_t{1} << 31))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %lld too large per SM",
+                static_cast<long long>(tiles), static_cast<long long>(row_len));
+  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  return SPARVAR_OK;
+}
+
+template <int D>
+int launch_decision_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to, const sparvar::dec::Args& a,
+                           cudaStream_t stream) {
+  auto kern = sparvar::dec::decision_attn_kernel<D>;
+  const uint32_t smem = sparvar::dec::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -156,9 +185,9 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   cudaFuncAttributes fa{};
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-  if (fa.numRegs != sparvar::fwd::kLaunchRegs)
-    return fail(SPARVAR_ERR_UNSUPPORTED, "attn_fwd_kernel compiled with %d registers per thread, "
-                "its register budgets assume %d", fa.numRegs, sparvar::fwd::kLaunchRegs);
+  if (fa.numRegs != sparvar::dec::kLaunchRegs)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "decision_attn_kernel compiled with %d registers per "
+                "thread, its register budgets assume %d", fa.numRegs, sparvar::dec::kLaunchRegs);
   // persistent: one CTA per SM, claiming the pairs blockIdx.x, blockIdx.x + gridDim.x, ...
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
@@ -167,14 +196,12 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   const int64_t pairs = a.total_pairs;
   const int64_t grid = pairs < sms ? pairs : sms;
   // the kernel's per-CTA sequence counters (blocks, ring loads) are 32-bit
-  int64_t row_len = 0;
-  for (int i = 0; i < a.n_problems; ++i) row_len = std::max<int64_t>(row_len, a.prob[i].idx_row_len);
-  if (ceil_div(pairs, grid) * (8 * row_len + 8) >= (int64_t{1} << 31))
-    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tile pairs x idx_row_len %lld too large per SM",
-                static_cast<long long>(pairs), static_cast<long long>(row_len));
-  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
+  if (ceil_div(pairs, grid) * (8 * static_cast<int64_t>(a.nkb) + 8) >= (int64_t{1} << 31))
+    return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tile pairs too many per SM",
+                static_cast<long long>(pairs));
+  kern<<<static_cast<unsigned>(grid), sparvar::dec::kThreads, smem, stream>>>(tq, tk, tv, to, a);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "decision_attn_kernel launch");
   return SPARVAR_OK;
 }
 
@@ -427,11 +454,11 @@ static int attn_fwd_prepare(FwdLaunch* L, const void* q, const void* k, const vo
   pr.Lq = Lq; pr.Lkv = Lkv;
   pr.nqb = static_cast<int>(ceil_div(Lq, 128));
   pr.nkb = static_cast<int>(ceil_div(Lkv, 128));
-  pr.q_row0 = 0; pr.pair0 = 0;
+  pr.q_row0 = 0; pr.tile0 = 0;
   pr.kv_cnt = kv_cnt; pr.kv_idx = kv_idx;
   pr.list_sb = list_strides[0]; pr.list_sh = list_strides[1];
   pr.idx_row_len = idx_row_len;
-  a.total_pairs = static_cast<int>(static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2));
+  a.total_tiles = static_cast<int>(static_cast<int64_t>(B) * H * pr.nqb);
   a.tile_mask = tile_mask;
   a.mask_shift = mask_shift;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -447,8 +474,7 @@ static int attn_fwd_prepare(FwdLaunch* L, const void* q, const void* k, const vo
     return rc;
   if ((rc = make_tmap(&L->tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v")))
     return rc;
-  if ((rc = make_tmap(&L->to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o",
-                      sparvar::fwd::kOutBoxRows)))
+  if ((rc = make_tmap(&L->to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o")))
     return rc;
   L->D = D;
   L->tok = tok != nullptr;
@@ -562,7 +588,7 @@ int sparvar_block_sparse_attn_fwd_multi(
   sparvar::fwd::Args a{};
   a.B = B; a.H = H; a.n_problems = n_problems;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  int64_t pairs = 0;
+  int64_t tiles = 0;
   for (int i = 0; i < n_problems; ++i) {
     if (q_row0[i] < 0 || lq[i] < 1 || static_cast<int64_t>(q_row0[i]) + lq[i] > q_rows)
       return fail(SPARVAR_ERR_INVALID_ARG, "problem %d: query rows [%d, %d + %d) outside [0, %d)", i,
@@ -577,15 +603,15 @@ int sparvar_block_sparse_attn_fwd_multi(
     pr.nqb = static_cast<int>(ceil_div(lq[i], 128));
     pr.nkb = static_cast<int>(ceil_div(lkv[i], 128));
     pr.q_row0 = q_row0[i];
-    pr.pair0 = static_cast<int>(pairs);
+    pr.tile0 = static_cast<int>(tiles);
     pr.kv_cnt = kv_cnt[i]; pr.kv_idx = kv_idx[i];
     pr.list_sb = list_strides[2 * i]; pr.list_sh = list_strides[2 * i + 1];
     pr.idx_row_len = idx_row_len[i];
-    pairs += static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2);
-    if (pairs > (int64_t{1} << 30))
-      return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tile pairs");
+    tiles += static_cast<int64_t>(B) * H * pr.nqb;
+    if (tiles > (int64_t{1} << 30))
+      return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
   }
-  a.total_pairs = static_cast<int>(pairs);
+  a.total_tiles = static_cast<int>(tiles);
   a.tile_mask = nullptr;
   a.mask_shift = 7;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -606,7 +632,7 @@ int sparvar_block_sparse_attn_fwd_multi(
     // the problem's own rows only, so the last tile's rows past its end are clipped
     const void* base = static_cast<const __nv_bfloat16*>(o) + q_row0[i] * o_strides[2];
     if ((rc = make_tmap(&to.m[i], base, D, lq[i], H, B, o_strides[2], o_strides[1], o_strides[0],
-                        "o", sparvar::fwd::kOutBoxRows)))
+                        "o")))
       return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -704,9 +730,9 @@ int sparvar_decision_attn_fwd(const void* q, const void* k, const void* v, void*
   if (Lq < 1 || Lkv < 1 || Lq > (1 << 30) || Lkv > (1 << 30))
     return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d Lkv=%d outside [1, 2^30]", Lq, Lkv);
   const int nkb = static_cast<int>(ceil_div(Lkv, 128));
-  if (nkb > sparvar::fwd::kMaxDecBlocks)
+  if (nkb > sparvar::dec::kMaxDecBlocks)
     return fail(SPARVAR_ERR_UNSUPPORTED, "Lkv=%d gives %d KV blocks (max %d)", Lkv, nkb,
-                sparvar::fwd::kMaxDecBlocks);
+                sparvar::dec::kMaxDecBlocks);
   if (static_cast<int64_t>(B) * H * ceil_div(Lq, 128) > (int64_t{1} << 30))
     return fail(SPARVAR_ERR_UNSUPPORTED, "B*H*ceil(Lq/128) above 2^30 query tiles");
   int rc;
@@ -721,21 +747,15 @@ int sparvar_decision_attn_fwd(const void* q, const void* k, const void* v, void*
   if (!(topk_ratio >= 0.f && topk_ratio <= 1.f))
     return fail(SPARVAR_ERR_INVALID_ARG, "topk_ratio must be in [0, 1] (0: mass threshold)");
 
-  sparvar::fwd::Args a{};
-  a.B = B; a.H = H; a.n_problems = 1;
+  sparvar::dec::Args a{};
+  a.B = B; a.H = H; a.Lq = Lq; a.Lkv = Lkv;
+  a.nqb = static_cast<int>(ceil_div(Lq, 128));
+  a.nkb = nkb;
+  a.total_pairs = static_cast<int>(static_cast<int64_t>(B) * H * ((a.nqb + 1) / 2));
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  sparvar::fwd::Problem& pr = a.prob[0];
-  pr.Lq = Lq; pr.Lkv = Lkv;
-  pr.nqb = static_cast<int>(ceil_div(Lq, 128));
-  pr.nkb = nkb;
-  pr.q_row0 = 0; pr.pair0 = 0;
-  pr.idx_row_len = nkb;
-  a.total_pairs = static_cast<int>(static_cast<int64_t>(B) * H * ((pr.nqb + 1) / 2));
-  a.mask_shift = 7;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.o_sb = o_strides[0]; a.o_sh = o_strides[1]; a.o_sr = o_strides[2];
   a.lse = lse;
-  a.lse_rows = Lq;
   a.dev_status = dev_status;
   a.mass_out = mass;
   a.mass_threshold = mass_threshold;
@@ -746,17 +766,16 @@ int sparvar_decision_attn_fwd(const void* q, const void* k, const void* v, void*
                : 0;
   a.sel_cnt = kv_cnt;
   a.sel_idx = kv_idx;
-  CUtensorMap tq, tk, tv;
-  sparvar::fwd::OutMaps to{};
+  CUtensorMap tq, tk, tv, to;
   if ((rc = make_tmap(&tq, q, D, Lq, H, B, q_strides[2], q_strides[1], q_strides[0], "q"))) return rc;
   if ((rc = make_tmap(&tk, k, D, Lkv, H, B, k_strides[2], k_strides[1], k_strides[0], "k"))) return rc;
   if ((rc = make_tmap(&tv, v, D, Lkv, H, B, v_strides[2], v_strides[1], v_strides[0], "v"))) return rc;
-  if ((rc = make_tmap(&to.m[0], o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o",
-                      sparvar::fwd::kOutBoxRows)))
+  if ((rc = make_tmap(&to, o, D, Lq, H, B, o_strides[2], o_strides[1], o_strides[0], "o",
+                      sparvar::dec::kOutBoxRows)))
     return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_fwd_kernel<128, false, false, true>(tq, tk, tv, to, a, st);
-  return launch_fwd_kernel<64, false, false, true>(tq, tk, tv, to, a, st);
+  if (D == 128) return launch_decision_kernel<128>(tq, tk, tv, to, a, st);
+  return launch_decision_kernel<64>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_ocache_apply(const void* o_target, const void* o_dense, const void* o_sparse, void* out,
