@@ -99,6 +99,7 @@ struct Args {
   float scale_log2;  // softmax_scale * log2(e)
   Problem prob[kMaxProblems];
   const uint64_t* tile_mask;  // per list entry, fine-block bits; null: whole tiles
+  const int32_t* tile_order;  // single problem: tile id at each position; null: in order
   int mask_shift;             // log2 of the fine block side (4, 5 or 6)
   __nv_bfloat16* o;
   int64_t o_sb, o_sh, o_sr;
@@ -141,7 +142,9 @@ struct Layout {
 // stream.  Any other non-empty tile starts with a prologue group (its first
 // score MMAs, issued once the predecessor's MMAs are done).
 struct TileCursor {
-  int t;  // tile id (problem tile0 + (b * H + h) * nqb + qb); >= total when the CTA is done
+  int t;  // position in the launch's tile sequence: the tile id (problem tile0 + (b * H + h) *
+          // nqb + qb), or for a single problem given an order, its index into that
+          // order; >= total when the CTA is done
   int p;  // problem of the tile
   int n;  // list length (clamped to [0, idx_row_len])
   const int32_t* list;
@@ -164,7 +167,8 @@ __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
     while (p + 1 < a.n_problems && t >= a.prob[p + 1].tile0) ++p;
   }
   const int nqb = a.prob[p].nqb;
-  const int lt = MULTI ? t - a.prob[p].tile0 : t;  // a single problem starts at tile 0, row 0
+  // a single problem starts at tile 0, row 0; its tiles may run in a given order
+  const int lt = MULTI ? t - a.prob[p].tile0 : (a.tile_order ? __ldg(a.tile_order + t) : t);
   const int bh = lt / nqb;
   return TileCoord{p, bh / a.H, bh % a.H, lt % nqb, a.prob[p].nkb, MULTI ? a.prob[p].q_row0 : 0};
 }

@@ -370,4 +370,61 @@ __global__ void validate_lists_kernel(const int32_t* kv_cnt, const int32_t* kv_i
   if (lane == 0 && flags) atomicOr(dev_status, flags);
 }
 
+// Order of the query tiles for the persistent attention kernel: longest lists
+// first, dealt to the kernel's G CTAs in a serpentine (round i of G tiles goes to
+// CTAs 0..G-1 when i is even and G-1..0 when i is odd), so that each CTA's total
+// work is close to the mean.  The kernel's CTA c takes the tiles at positions
+// c, c + G, c + 2G, ... of `order`.  Tile id = (b * H + h) * nqb + qb.  One CTA:
+// a histogram of the list lengths (clamped to kOrderBuckets - 1; ties in any
+// order), a scan for each length's first position, then one position per tile.
+constexpr int kOrderBuckets = 1024;
+__global__ void __launch_bounds__(1024)
+    tile_order_kernel(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H, int nqb,
+                      int idx_row_len, int G, int32_t* order) {
+  __shared__ int hist[kOrderBuckets];
+  __shared__ int warp_sum[32];
+  const int T = B * H * nqb;
+  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  auto bucket = [&](int t) {
+    const int qb = t % nqb, bh = t / nqb;
+    int n = __ldg(kv_cnt + (bh / H) * sb + (bh % H) * sh + qb);
+    n = n < 0 ? 0 : (n > idx_row_len ? idx_row_len : n);
+    return kOrderBuckets - 1 - (n < kOrderBuckets - 1 ? n : kOrderBuckets - 1);  // longest first
+  };
+  for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[bucket(t)], 1);
+  __syncthreads();
+  // exclusive scan of the histogram (blockDim.x == kOrderBuckets: one bucket each)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int h = hist[threadIdx.x];
+  int x = h;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int v = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    warp_sum[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  const int start = x - h + (w > 0 ? warp_sum[w - 1] : 0);
+  __syncthreads();
+  hist[threadIdx.x] = start;
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int pos = atomicAdd(&hist[bucket(t)], 1);  // the tile's rank, longest first
+    const int r = pos / G, j = pos % G;
+    const int in_round = min(G, T - r * G);
+    order[r * G + ((r & 1) ? in_round - 1 - j : j)] = t;
+  }
+}
+
 }  // namespace sparvar

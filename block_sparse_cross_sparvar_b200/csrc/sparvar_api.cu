@@ -537,14 +537,61 @@ static int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, f
                          const int64_t* list_strides, int idx_row_len, const uint64_t* tile_mask,
                          int mask_block, int block_q, int block_kv, float softmax_scale,
                          int32_t* dev_status, void* stream,
-                         const sparvar::fwd::CslaTokens* tok) {
+                         const sparvar::fwd::CslaTokens* tok,
+                         const int32_t* tile_order = nullptr) {
   FwdLaunch L;
   int rc = attn_fwd_prepare(&L, q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides,
                             v_strides, o_strides, kv_cnt, kv_idx, list_strides, idx_row_len,
                             tile_mask, mask_block, block_q, block_kv, softmax_scale, dev_status,
                             tok);
   if (rc) return rc;
+  L.a.tile_order = tile_order;
   return attn_fwd_launch(L, stream);
+}
+
+// the persistent attention kernel's grid for T query tiles on the current device
+static int attn_grid(int64_t T, int* grid) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
+  *grid = static_cast<int>(T < sms ? T : sms);
+  return SPARVAR_OK;
+}
+
+int sparvar_tile_order(const int32_t* kv_cnt, int B, int H, int Lq,
+                       const int64_t* list_strides, int idx_row_len, int32_t* order,
+                       void* stream) {
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (Lq < 1 || Lq > (1 << 30)) return fail(SPARVAR_ERR_INVALID_ARG, "Lq=%d outside [1, 2^30]", Lq);
+  if (!kv_cnt || !order || !list_strides || list_strides[0] < 0 || list_strides[1] < 0 ||
+      idx_row_len < 0)
+    return fail(SPARVAR_ERR_INVALID_ARG, "bad lists or order buffer");
+  const int64_t nqb = ceil_div(Lq, 128);
+  const int64_t T = static_cast<int64_t>(B) * H * nqb;
+  if (T > (int64_t{1} << 30)) return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
+  int G = 0, rc;
+  if ((rc = attn_grid(T, &G))) return rc;
+  sparvar::tile_order_kernel<<<1, sparvar::kOrderBuckets, 0, static_cast<cudaStream_t>(stream)>>>(
+      kv_cnt, list_strides[0], list_strides[1], B, H, static_cast<int>(nqb), idx_row_len, G, order);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tile_order_kernel launch");
+  return SPARVAR_OK;
+}
+
+int sparvar_block_sparse_attn_fwd_ordered(const void* q, const void* k, const void* v, void* o,
+                                          float* lse, int B, int H, int Lq, int Lkv, int D,
+                                          const int64_t* q_strides, const int64_t* k_strides,
+                                          const int64_t* v_strides, const int64_t* o_strides,
+                                          const int32_t* kv_cnt, const int32_t* kv_idx,
+                                          const int64_t* list_strides, int idx_row_len,
+                                          const int32_t* tile_order, float softmax_scale,
+                                          int32_t* dev_status, void* stream) {
+  if (!tile_order) return fail(SPARVAR_ERR_INVALID_ARG, "tile_order is NULL");
+  return attn_fwd_impl(q, k, v, o, lse, B, H, Lq, Lkv, D, q_strides, k_strides, v_strides,
+                       o_strides, kv_cnt, kv_idx, list_strides, idx_row_len, nullptr, 0, 128, 128,
+                       softmax_scale, dev_status, stream, nullptr, tile_order);
 }
 
 int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,

@@ -39,6 +39,10 @@ EXPORTS = {
     "sparvar_block_sparse_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p, _i64p,
                                        _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _i, _i, _i, _f, _vp,
                                        _vp], _i),
+    "sparvar_tile_order": ([_vp, _i, _i, _i, _i64p, _i, _vp, _vp], _i),
+    "sparvar_block_sparse_attn_fwd_ordered": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
+                                               _i64p, _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _f,
+                                               _vp, _vp], _i),
     "sparvar_map_indices_2d": ([_vp, _vp, _i, _i, _i32p, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                 _vp, _vp], _i),
     "sparvar_block_sparse_attn_fwd_static": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
@@ -176,12 +180,35 @@ def sparvar_coarsen_lists(kv_cnt, kv_idx, B, H, Lq, Lkv, block, dev_status=None)
     return t_cnt, t_idx, t_mask
 
 
+def sparvar_tile_order(kv_cnt, B, H, Lq, out=None):
+    """Query tiles longest list first, dealt in a serpentine to the attention
+    kernel's CTAs (lists over 128x128 blocks): int32 [B * H * ceil(Lq / 128)]."""
+    if kv_cnt.dtype != torch.int32:
+        raise SparvarError("kv_cnt must be int32")
+    nqb = -(-Lq // 128)
+    if kv_cnt.shape[-1] != nqb:
+        raise SparvarError(f"kv_cnt has {kv_cnt.shape[-1]} query blocks, expected {nqb}")
+    T = B * H * nqb
+    if out is None:
+        out = torch.empty(T, dtype=torch.int32, device=kv_cnt.device)
+    if out.dtype != torch.int32 or out.numel() != T or not out.is_contiguous():
+        raise SparvarError(f"out must be a contiguous int32 tensor of {T} elements")
+    sb, sh = _list_strides(kv_cnt, B, H)
+    # counts are only ranked here (the attention call checks them against its lists)
+    _check(lib().sparvar_tile_order(_ptr(kv_cnt), B, H, Lq, _i64([sb, sh]), 1 << 30, _ptr(out),
+                                    _stream(kv_cnt.device)), "sparvar_tile_order")
+    return out
+
+
 def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv=128,
-                                  softmax_scale=None, out=None, return_lse=False, dev_status=None):
+                                  softmax_scale=None, out=None, return_lse=False, dev_status=None,
+                                  tile_order=None):
     """Block-sparse attention forward: returns O (and the row LSE when asked).
 
     Lists over 128x128 blocks go to the kernel as they are; lists over square
-    16/32/64 blocks are first coarsened to 128x128 tiles with per-tile masks."""
+    16/32/64 blocks are first coarsened to 128x128 tiles with per-tile masks.
+    ``tile_order`` (from sparvar_tile_order on the same lists; 128x128 blocks only)
+    sets the order in which the kernel's CTAs take the query tiles."""
     B, H, Lq, D = q.shape
     Lkv = k.shape[2]
     if k.shape != (B, H, Lkv, D) or v.shape != (B, H, Lkv, D):
@@ -207,6 +234,17 @@ def sparvar_block_sparse_attn_fwd(q, k, v, kv_cnt, kv_idx, block_q=128, block_kv
     lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device) if return_lse else None
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     sb, sh = _list_strides(kv_cnt, B, H)
+    if tile_order is not None:
+        if tile_mask is not None:
+            raise SparvarError("tile_order needs lists over 128x128 blocks")
+        if (tile_order.dtype != torch.int32 or tile_order.numel() != B * H * nqb
+                or not tile_order.is_contiguous()):
+            raise SparvarError(f"tile_order must be a contiguous int32 tensor of {B * H * nqb}")
+        _check(lib().sparvar_block_sparse_attn_fwd_ordered(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
+            _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], _ptr(tile_order), scale,
+            _ptr(dev_status), _stream(q.device)), "sparvar_block_sparse_attn_fwd_ordered")
+        return (out, lse) if return_lse else out
     _check(lib().sparvar_block_sparse_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Lq, Lkv, D, qs, ks, vs, os_,
         _ptr(kv_cnt), _ptr(kv_idx), _i64([sb, sh]), kv_idx.shape[-1], _ptr(tile_mask), mask_block,

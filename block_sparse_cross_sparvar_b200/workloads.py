@@ -12,7 +12,8 @@
   64x64 blocks and the token mask inside 128x128 tiles.
 * ``density_sweep``: the last scale with random block lists at fixed densities
   (sink block always kept), with the full key prefix and with the 40x40 and
-  48x48 scales skipped from the prefix.
+  48x48 scales skipped from the prefix; each also with the query tiles taken
+  longest list first.
 
 Every step runs in the library's kernels; torch only provides memory, streams
 and events.
@@ -327,8 +328,15 @@ def density_sweep(device, reps=10, seed=0, B=2, H=16, D=128, densities=(0.05, 0.
                         idx_np[bb, hh, qb, :kept.size] = kept
             idx = torch.from_numpy(idx_np).to(device)
             ms = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, out=out), reps, device)
+            # the same lists with the query tiles taken longest list first; the order is
+            # built inside the timed call
+            order = torch.empty(B * H * nqb, dtype=torch.int32, device=device)
+            ms_lpt = time_ms(lambda: ops.sparvar_block_sparse_attn_fwd(
+                q, k, v, cnt, idx, out=out,
+                tile_order=ops.sparvar_tile_order(cnt, B, H, 4096, out=order)), reps, device)
             f, _ = kept_flops(cnt, idx, 4096, L, 128, D)
             res.append({"prefix": name, "Lkv": L, "target_density": dens,
                         "density": f / (4 * 4096 * L * D * B * H), "ms": ms,
-                        "tflops": f / (ms * 1e-3) / 1e12})
+                        "tflops": f / (ms * 1e-3) / 1e12, "ms_longest_first": ms_lpt,
+                        "tflops_longest_first": f / (ms_lpt * 1e-3) / 1e12})
     return {"workload": "last_scale_density_sweep", "B": B, "H": H, "D": D, "runs": res}

@@ -267,6 +267,36 @@ SPARVAR_API int sparvar_block_sparse_attn_fwd(const void* q, const void* k, cons
                                   void* stream);
 
 /*
+ * Longest lists first (a scheduling aid for the persistent attention kernel; the
+ * pages fix no tile order): writes into order[T], T = B * H * ceil(Lq / 128), the
+ * tile ids (b * H + h) * nqb + qb sorted by list length, longest first, then dealt
+ * to the kernel's G = min(T, SMs of the current device) CTAs in a serpentine
+ * (round i of G tiles to CTAs 0..G-1 for even i, G-1..0 for odd i), so that each
+ * CTA's total list length is close to the mean.  Lengths above 1022 count as 1023;
+ * ties are taken in any order.  kv_cnt, list_strides and idx_row_len as for
+ * sparvar_block_sparse_attn_fwd with 128x128 blocks; order is device int32 owned
+ * by the caller.  One launch of one CTA on `stream`; the order depends on the
+ * device's SM count, so it is for launches on that device.  Errors: a bad shape
+ * or pointer is refused before anything is enqueued.
+ */
+SPARVAR_API int sparvar_tile_order(const int32_t* kv_cnt, int B, int H, int Lq,
+                                   const int64_t* list_strides, int idx_row_len, int32_t* order,
+                                   void* stream);
+
+/*
+ * sparvar_block_sparse_attn_fwd over 128x128 block lists (no tile mask), the
+ * kernel's CTAs taking the query tiles in the order written by sparvar_tile_order
+ * for the same lists and device (tile_order, device int32 [T], not NULL).  The
+ * result does not depend on the order; only the balance of the CTAs' work does.
+ */
+SPARVAR_API int sparvar_block_sparse_attn_fwd_ordered(
+    const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq,
+    int Lkv, int D, const int64_t* q_strides, const int64_t* k_strides, const int64_t* v_strides,
+    const int64_t* o_strides, const int32_t* kv_cnt, const int32_t* kv_idx,
+    const int64_t* list_strides, int idx_row_len, const int32_t* tile_order, float softmax_scale,
+    int32_t* dev_status, void* stream);
+
+/*
  * Fine block lists to 128x128 tile lists with per-tile bitmasks, the form the
  * attention call takes for block sizes below 128 ("Main Findings" block-size
  * rows: the mask is defined on a fine grid, the contraction runs on 128x128

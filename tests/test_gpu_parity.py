@@ -69,15 +69,18 @@ def test_csla_every_scale_and_block_size():
 
 
 # ------------------------------------------------------------------ attention
-def _check_attention(q_bits, k_bits, v_bits, blk_lists, bq, bk, D, lse_check=True, scale=None):
-    """q/k/v bits [B,H,*,D]; blk_lists = (cnt, idx) torch (shared or per (b,h))."""
+def _check_attention(q_bits, k_bits, v_bits, blk_lists, bq, bk, D, lse_check=True, scale=None,
+                     ordered=False):
+    """q/k/v bits [B,H,*,D]; blk_lists = (cnt, idx) torch (shared or per (b,h));
+    ordered: the kernel takes the query tiles longest list first."""
     B, H, Lq, _ = q_bits.shape
     Lkv = k_bits.shape[2]
     q, k, v = _dev(q_bits), _dev(k_bits), _dev(v_bits)
     cnt, idx = blk_lists
     st = _status()
+    order = ops.sparvar_tile_order(cnt, B, H, Lq) if ordered else None
     o, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, bq, bk, softmax_scale=scale,
-                                               return_lse=True, dev_status=st)
+                                               return_lse=True, dev_status=st, tile_order=order)
     torch.cuda.synchronize()
     assert st.item() == 0
     o = o.float().cpu().numpy()
@@ -271,6 +274,64 @@ def test_attention_persistent_short_and_empty_lists(D):
     cnt = torch.from_numpy(lens.astype(np.int32)).cuda()
     idx = torch.from_numpy(idx_np).cuda()
     _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D)
+
+
+def test_tile_order_longest_first_serpentine():
+    """The order is a permutation of the tiles; round r of G positions holds the r-th
+    G longest lists (longest first over the whole order), dealt to CTAs 0..G-1 for
+    even r and G-1..0 for odd r."""
+    rng = np.random.default_rng(5)
+    B, H, nqb = 2, 16, 40
+    lens = rng.integers(0, 30, size=(B, H, nqb)).astype(np.int32)
+    cnt = torch.from_numpy(lens).cuda()
+    order = ops.sparvar_tile_order(cnt, B, H, nqb * 128).cpu().numpy()
+    T = B * H * nqb
+    G = min(T, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert sorted(order.tolist()) == list(range(T))
+    flat = lens.reshape(-1)
+    ranked = np.sort(flat)[::-1]
+    for r in range(-(-T // G)):
+        pos = order[r * G:(r + 1) * G]
+        got = flat[pos]
+        # this round holds exactly the next lengths of the ranking
+        assert sorted(got.tolist()) == sorted(ranked[r * G:(r + 1) * G].tolist())
+        # and deals them longest first in its direction
+        seq = got if r % 2 == 0 else got[::-1]
+        assert all(seq[i] >= seq[i + 1] for i in range(len(seq) - 1))
+
+
+def test_attention_in_tile_order():
+    """Taking the query tiles longest first changes which CTA runs a tile and what
+    comes before it (and so which softmax group takes which of its blocks, and the
+    order in which the two groups' PVs add into O): the output matches the oracle
+    as in natural order, and the two agree to within rounding."""
+    rng = np.random.default_rng(23)
+    B, H, D = 2, 16, 128
+    nqb, nkb = 40, 6
+    Lq, Lkv = nqb * 128 - 37, nkb * 128 - 50
+    bits = {n: inputs.bf16_round(rng.standard_normal((B, H, L, D)).astype(np.float32))[0]
+            for n, L in (("q", Lq), ("k", Lkv), ("v", Lkv))}
+    lens = rng.choice(nkb + 1, size=(B, H, nqb), p=[0.15, 0.2, 0.2, 0.15, 0.1, 0.1, 0.1])
+    idx_np = np.full((B, H, nqb, nkb), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                idx_np[b, h, qb, :lens[b, h, qb]] = rng.permutation(nkb)[:lens[b, h, qb]]
+    cnt = torch.from_numpy(lens.astype(np.int32)).cuda()
+    idx = torch.from_numpy(idx_np).cuda()
+    q, k, v = _dev(bits["q"]), _dev(bits["k"]), _dev(bits["v"])
+    o1, l1 = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True)
+    order = ops.sparvar_tile_order(cnt, B, H, Lq)
+    st = _status()
+    o2, l2 = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True,
+                                               tile_order=order, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+    fin = torch.isfinite(l1)
+    assert torch.equal(fin, torch.isfinite(l2))
+    assert (l1[fin] - l2[fin]).abs().max().item() < 1e-4
+    _check_attention(bits["q"], bits["k"], bits["v"], (cnt, idx), 128, 128, D, ordered=True)
 
 
 def test_attention_unordered_lists_give_same_result():

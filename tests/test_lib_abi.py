@@ -185,3 +185,32 @@ def test_wait_probe_rejects_bad_arguments(lib):
     assert lib.sparvar_wait_timeout_probe(999, vp(16), vp(16), vp(0)) == 1
     assert "limit_ns=999" in lib.sparvar_last_error().decode()
     assert lib.sparvar_wait_timeout_probe(10**9 + 1, vp(16), vp(16), vp(0)) == 1
+
+
+def test_tile_order_rejects_bad_arguments(lib):
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    vp = ctypes.c_void_p
+    cases = [((vp(0), 1, 1, 128, i64(0, 0), 1, vp(16), vp(0)), "bad lists"),
+             ((vp(16), 1, 1, 128, i64(0, 0), 1, vp(0), vp(0)), "bad lists"),
+             ((vp(16), 0, 1, 128, i64(0, 0), 1, vp(16), vp(0)), "B=0"),
+             ((vp(16), 1, 1, 0, i64(0, 0), 1, vp(16), vp(0)), "Lq=0"),
+             ((vp(16), 1, 1, 128, i64(-1, 0), 1, vp(16), vp(0)), "bad lists")]
+    for args, msg in cases:
+        assert lib.sparvar_tile_order(*args) == 1
+        assert msg in lib.sparvar_last_error().decode()
+
+
+def test_ordered_attention_rejects_bad_arguments(lib):
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)  # noqa: E731
+    vp = ctypes.c_void_p
+
+    def call(order, D=128):
+        return lib.sparvar_block_sparse_attn_fwd_ordered(
+            vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 128, 128, D, i64(0, 0, 128),
+            i64(0, 0, 128), i64(0, 0, 128), i64(0, 0, 128), vp(16), vp(16), i64(0, 0), 1,
+            vp(order), ctypes.c_float(0.1), vp(0), vp(0))
+
+    assert call(0) == 1
+    assert "tile_order is NULL" in lib.sparvar_last_error().decode()
+    assert call(16, D=96) == 2
+    assert "D=96" in lib.sparvar_last_error().decode()

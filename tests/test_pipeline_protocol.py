@@ -340,3 +340,15 @@ def test_ring_wait_before_p_is_caught():
             assert "parity ambiguity" in str(e)
             caught += 1
     assert caught > 0
+
+
+def test_longest_first_orders():
+    """The kernel can take its tiles longest list first (a serpentine over the CTAs);
+    a CTA then walks its lengths in falling order, with empty tiles last.  Such
+    sequences, and the same lengths rising, run clean."""
+    rng = random.Random(11)
+    for t in range(40):
+        tiles = [rng.choice([0, 0, 1, 2, 3, 4, 6, 9]) for _ in range(rng.randint(2, 8))]
+        for seq in (sorted(tiles, reverse=True), sorted(tiles)):
+            for ns in (5, 6):
+                assert Model(seq, ns, 0.3, t).run(), (seq, ns)
