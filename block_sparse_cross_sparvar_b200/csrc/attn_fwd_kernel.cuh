@@ -99,7 +99,7 @@ struct Args {
   float scale_log2;  // softmax_scale * log2(e)
   Problem prob[kMaxProblems];
   const uint64_t* tile_mask;  // per list entry, fine-block bits; null: whole tiles
-  const int32_t* tile_order;  // single problem: tile id at each position; null: in order
+  const int32_t* tile_order;  // ORD instantiation: the tile id at each position
   int mask_shift;             // log2 of the fine block side (4, 5 or 6)
   __nv_bfloat16* o;
   int64_t o_sb, o_sh, o_sr;
@@ -160,23 +160,28 @@ struct TileCoord {
   int p, b, h, qb;
   int nkb, row0;  // the problem's key-block count and first query row
 };
-template <bool MULTI>
+// How a launch numbers its tiles: one problem in natural order, several
+// problems (a problem table), or one problem in a given order (args.tile_order).
+constexpr int kSingle = 0, kProblems = 1, kOrdered = 2;
+template <int PM>
 __device__ __forceinline__ TileCoord tile_coord(int t, const Args& a) {
   int p = 0;
-  if constexpr (MULTI) {
+  if constexpr (PM == kProblems) {
     while (p + 1 < a.n_problems && t >= a.prob[p + 1].tile0) ++p;
   }
   const int nqb = a.prob[p].nqb;
   // a single problem starts at tile 0, row 0; its tiles may run in a given order
-  const int lt = MULTI ? t - a.prob[p].tile0 : (a.tile_order ? __ldg(a.tile_order + t) : t);
+  const int lt = PM == kProblems ? t - a.prob[p].tile0
+                                 : (PM == kOrdered ? __ldg(a.tile_order + t) : t);
   const int bh = lt / nqb;
-  return TileCoord{p, bh / a.H, bh % a.H, lt % nqb, a.prob[p].nkb, MULTI ? a.prob[p].q_row0 : 0};
+  return TileCoord{p, bh / a.H, bh % a.H, lt % nqb, a.prob[p].nkb,
+                   PM == kProblems ? a.prob[p].q_row0 : 0};
 }
 
-template <bool MULTI>
+template <int PM>
 __device__ __forceinline__ int tile_count(int t, const Args& a, bool report,
                                           const int32_t** list, int* prob) {
-  const TileCoord tc = tile_coord<MULTI>(t, a);
+  const TileCoord tc = tile_coord<PM>(t, a);
   const Problem& pr = a.prob[tc.p];
   const int64_t lrow = tc.b * pr.list_sb + tc.h * pr.list_sh + tc.qb;
   int n = __ldg(pr.kv_cnt + lrow);
@@ -189,13 +194,13 @@ __device__ __forceinline__ int tile_count(int t, const Args& a, bool report,
   return n;
 }
 
-template <bool MULTI>
+template <int PM>
 __device__ __forceinline__ void cursor_load(TileCursor& c, const Args& a, int total, bool report) {
   if (c.t >= total) return;
-  c.n = tile_count<MULTI>(c.t, a, report, &c.list, &c.p);
+  c.n = tile_count<PM>(c.t, a, report, &c.list, &c.p);
   c.next_n = 0;
   for (int t = c.t + gridDim.x; t < total && c.next_n == 0; t += gridDim.x)
-    c.next_n = tile_count<MULTI>(t, a, false, nullptr, nullptr);
+    c.next_n = tile_count<PM>(t, a, false, nullptr, nullptr);
 }
 
 __device__ __forceinline__ bool has_prologue(const TileCursor& c) { return c.prev_n < 3; }
@@ -224,7 +229,7 @@ __device__ __forceinline__ int group_of_block(const TileCursor& c, int j) {
   return c.G + (has_prologue(c) ? 1 : 0) + j;
 }
 
-template <bool MULTI>
+template <int PM>
 __device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int total, bool report) {
   if (c.n > 0) {
     c.pos0 += ring_items(c);
@@ -234,7 +239,7 @@ __device__ __forceinline__ void cursor_next(TileCursor& c, const Args& a, int to
     c.prev_n = c.n;
   }
   c.t += gridDim.x;
-  cursor_load<MULTI>(c, a, total, report);
+  cursor_load<PM>(c, a, total, report);
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -296,12 +301,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // TOK: apply the CSLA token mask (args.tok) inside the kept tiles.  MULTI: the
 // launch holds several problems (args.prob), one output map each.
-template <int D, bool TOK, bool MULTI>
+template <int D, bool TOK, bool MULTI, bool ORD = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ OutMaps tm_os, const __grid_constant__ Args args) {
+  constexpr int PM = MULTI ? kProblems : (ORD ? kOrdered : kSingle);
   using L = Layout<D>;
   constexpr int NS = L::kSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileCursor first{};
   first.t = blockIdx.x;
   first.prev_n = -1;
-  cursor_load<MULTI>(first, args, total, threadIdx.x == 0);
+  cursor_load<PM>(first, args, total, threadIdx.x == 0);
 
   if (warp == kLoadWarp) {
     // ================================================================ producer
@@ -398,9 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       tq.row0 + tq.qb * kTile, tq.h, tq.b);
         if (qs) ++q_issued1; else ++q_issued0;
       };
-      for (TileCursor c = first; c.t < total && ok; cursor_next<MULTI>(c, args, total, false)) {
+      for (TileCursor c = first; c.t < total && ok; cursor_next<PM>(c, args, total, false)) {
         if (c.n == 0) continue;
-        const TileCoord tc = tile_coord<MULTI>(c.t, args);
+        const TileCoord tc = tile_coord<PM>(c.t, args);
         if (has_prologue(c)) {
           load_q(c.k, tc);
           for (int jj = 0; jj < n_prologue(c) && ok; ++jj)
@@ -411,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileCoord tn{};
         if (feeds_next(c)) {
           do {
-            cursor_next<MULTI>(nx, args, total, false);
+            cursor_next<PM>(nx, args, total, false);
           } while (nx.t < total && nx.n == 0);
-          tn = tile_coord<MULTI>(nx.t, args);
+          tn = tile_coord<PM>(nx.t, args);
         }
         const int nk = own_k(c);
         for (int j = 0; j < c.n && ok; ++j) {
@@ -462,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       int last1 = -1, last2 = -1;  // last two groups of the previous non-empty tile
-      for (TileCursor c = first; c.t < total && ok; cursor_next<MULTI>(c, args, total, false)) {
+      for (TileCursor c = first; c.t < total && ok; cursor_next<PM>(c, args, total, false)) {
         if (c.n == 0) continue;
         const int nk = own_k(c);
         if (me == 0 && has_prologue(c)) {
@@ -528,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float csc = args.scale_log2;
     bool good = true;
 
-    for (TileCursor c = first; c.t < total; cursor_next<MULTI>(c, args, total, threadIdx.x == 0)) {
+    for (TileCursor c = first; c.t < total; cursor_next<PM>(c, args, total, threadIdx.x == 0)) {
       // the tile's problem, read once per tile into registers
       const int pi = MULTI ? c.p : 0;
       const int p_nkb = args.prob[pi].nkb, p_lkv = args.prob[pi].Lkv, p_lq = args.prob[pi].Lq;
@@ -746,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       tc_fence_after();
       const int aborted = __shfl_sync(0xffffffffu, *abort_flag, 0);
-      const TileCoord tc = tile_coord<MULTI>(c.t, args);
+      const TileCoord tc = tile_coord<PM>(c.t, args);
       const int grow = tc.qb * kTile + row;
       float l = 0.f, m = -INFINITY, inv_l = 0.f;
       if (c.n > 0) {
