@@ -66,6 +66,71 @@ __device__ __forceinline__ void compact_bitset(const uint32_t* bits, int nkb, in
   if (lane == 0) *cnt_out = base;
 }
 
+// Order of the query tiles for the persistent attention kernel: longest lists
+// first, dealt to the kernel's G CTAs in a serpentine (round i of G tiles goes to
+// CTAs 0..G-1 when i is even and G-1..0 when i is odd), so that each CTA's total
+// work is close to the mean.  The kernel's CTA c takes the tiles at positions
+// c, c + G, c + 2G, ... of `order`.  Tile id = (b * H + h) * nqb + qb.  One CTA:
+// a histogram of the list lengths (clamped to kOrderBuckets - 1; ties in any
+// order), a scan for each length's first position, then one position per tile.
+// The counts are read through L2 (they may have been written by other CTAs of
+// the same launch).
+constexpr int kOrderBuckets = 1024;
+__device__ void order_tiles_block(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H,
+                                  int nqb, int idx_row_len, int G, int32_t* order) {
+  __shared__ int hist[kOrderBuckets];
+  __shared__ int part[32];
+  const int T = B * H * nqb;
+  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  auto bucket = [&](int t) {
+    const int qb = t % nqb, bh = t / nqb;
+    int n = __ldcg(kv_cnt + (bh / H) * sb + (bh % H) * sh + qb);
+    n = n < 0 ? 0 : (n > idx_row_len ? idx_row_len : n);
+    return kOrderBuckets - 1 - (n < kOrderBuckets - 1 ? n : kOrderBuckets - 1);  // longest first
+  };
+  for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[bucket(t)], 1);
+  __syncthreads();
+  // exclusive scan of the histogram: each thread takes per = kOrderBuckets / blockDim.x
+  // consecutive buckets, then the threads' totals are scanned across warps
+  const int per = kOrderBuckets / blockDim.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int tot = 0;
+  for (int i = 0; i < per; ++i) tot += hist[threadIdx.x * per + i];
+  int x = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) part[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int v = lane < (blockDim.x >> 5) ? part[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    part[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  int start = x - tot + (w > 0 ? part[w - 1] : 0);
+  __syncthreads();
+  for (int i = 0; i < per; ++i) {
+    const int h = hist[threadIdx.x * per + i];
+    hist[threadIdx.x * per + i] = start;
+    start += h;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int pos = atomicAdd(&hist[bucket(t)], 1);  // the tile's rank, longest first
+    const int r = pos / G, j = pos % G;
+    const int in_round = min(G, T - r * G);
+    order[r * G + ((r & 1) ? in_round - 1 - j : j)] = t;
+  }
+}
+
 // ---------------------------------------------------------------- CSLA
 // For the query block's rows, each (query row i, scale m) pair contributes the
 // keys of scale m in rows [ci - r, ci + r] and columns [cl - r, ch + r], where
@@ -73,10 +138,19 @@ __device__ __forceinline__ void compact_bitset(const uint32_t* bits, int nkb, in
 // row i (the projection of consecutive columns moves by 0 or 1, so the union of
 // the per-query windows is that rectangle).  Each key row of the rectangle is a
 // contiguous token range, which sets a contiguous range of KV-block bits.
+// With `order` set, the CTA that finishes last (counted in *done, which it sets
+// back to zero) also writes the longest-first tile order of the lists for a
+// (B, H) launch of the attention kernel on G CTAs (the lists are shared by every
+// batch item and head).
+struct TileOrderOut {
+  int32_t* order;  // null: no order
+  int32_t* done;   // zero before the launch, zero after it
+  int B, H, G;
+};
 __global__ void __launch_bounds__(kMaskThreads)
     csla_mask_kernel(const ScaleGeometry g, int q_scale, int n_sink, int r_prev, int r_own,
                      int block_q, int block_kv, int nkb, int32_t* kv_cnt, int32_t* kv_idx,
-                     uint8_t* blk_mask) {
+                     uint8_t* blk_mask, const TileOrderOut ord) {
   extern __shared__ uint32_t bits[];
   const int qb = blockIdx.x;
   const int nwords = (nkb + 31) >> 5;
@@ -119,6 +193,18 @@ __global__ void __launch_bounds__(kMaskThreads)
   if (threadIdx.x < 32)
     compact_bitset(bits, nkb, kv_idx + static_cast<int64_t>(qb) * nkb, kv_cnt + qb,
                    blk_mask ? blk_mask + static_cast<int64_t>(qb) * nkb : nullptr);
+  if (ord.order) {
+    __shared__ int last;
+    __threadfence();  // this CTA's count is visible before it is counted as done
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(ord.done, 1) == static_cast<int>(gridDim.x) - 1;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      order_tiles_block(kv_cnt, 0, 0, ord.B, ord.H, gridDim.x, nkb, ord.G, ord.order);
+      if (threadIdx.x == 0) *ord.done = 0;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- CS4A mapping
@@ -370,61 +456,11 @@ __global__ void validate_lists_kernel(const int32_t* kv_cnt, const int32_t* kv_i
   if (lane == 0 && flags) atomicOr(dev_status, flags);
 }
 
-// Order of the query tiles for the persistent attention kernel: longest lists
-// first, dealt to the kernel's G CTAs in a serpentine (round i of G tiles goes to
-// CTAs 0..G-1 when i is even and G-1..0 when i is odd), so that each CTA's total
-// work is close to the mean.  The kernel's CTA c takes the tiles at positions
-// c, c + G, c + 2G, ... of `order`.  Tile id = (b * H + h) * nqb + qb.  One CTA:
-// a histogram of the list lengths (clamped to kOrderBuckets - 1; ties in any
-// order), a scan for each length's first position, then one position per tile.
-constexpr int kOrderBuckets = 1024;
+// The order on its own: one CTA of 1024 threads.
 __global__ void __launch_bounds__(1024)
     tile_order_kernel(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H, int nqb,
                       int idx_row_len, int G, int32_t* order) {
-  __shared__ int hist[kOrderBuckets];
-  __shared__ int warp_sum[32];
-  const int T = B * H * nqb;
-  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  auto bucket = [&](int t) {
-    const int qb = t % nqb, bh = t / nqb;
-    int n = __ldg(kv_cnt + (bh / H) * sb + (bh % H) * sh + qb);
-    n = n < 0 ? 0 : (n > idx_row_len ? idx_row_len : n);
-    return kOrderBuckets - 1 - (n < kOrderBuckets - 1 ? n : kOrderBuckets - 1);  // longest first
-  };
-  for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[bucket(t)], 1);
-  __syncthreads();
-  // exclusive scan of the histogram (blockDim.x == kOrderBuckets: one bucket each)
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int h = hist[threadIdx.x];
-  int x = h;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sum[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int v = warp_sum[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += y;
-    }
-    warp_sum[lane] = v;  // inclusive over warps
-  }
-  __syncthreads();
-  const int start = x - h + (w > 0 ? warp_sum[w - 1] : 0);
-  __syncthreads();
-  hist[threadIdx.x] = start;
-  __syncthreads();
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const int pos = atomicAdd(&hist[bucket(t)], 1);  // the tile's rank, longest first
-    const int r = pos / G, j = pos % G;
-    const int in_round = min(G, T - r * G);
-    order[r * G + ((r & 1) ? in_round - 1 - j : j)] = t;
-  }
+  order_tiles_block(kv_cnt, sb, sh, B, H, nqb, idx_row_len, G, order);
 }
 
 }  // namespace sparvar

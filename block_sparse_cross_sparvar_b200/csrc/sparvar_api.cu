@@ -228,9 +228,44 @@ int sparvar_scale_blocks(const int32_t* sides, int n_scales, int q_scale, int bl
   return SPARVAR_OK;
 }
 
+static int csla_mask_impl(const int32_t* sides, int n_scales, int q_scale, int n_sink_scales,
+                          int radius_prev, int radius_own, int block_q, int block_kv,
+                          int32_t* kv_cnt, int32_t* kv_idx, uint8_t* blk_mask, void* stream,
+                          sparvar::TileOrderOut ord);
+
 int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int q_scale, int n_sink_scales,
                             int radius_prev, int radius_own, int block_q, int block_kv,
                             int32_t* kv_cnt, int32_t* kv_idx, uint8_t* blk_mask, void* stream) {
+  return csla_mask_impl(sides, n_scales, q_scale, n_sink_scales, radius_prev, radius_own, block_q,
+                        block_kv, kv_cnt, kv_idx, blk_mask, stream,
+                        sparvar::TileOrderOut{nullptr, nullptr, 0, 0, 0});
+}
+
+static int attn_grid(int64_t T, int* grid);
+
+int sparvar_build_csla_mask_ordered(const int32_t* sides, int n_scales, int q_scale,
+                                    int n_sink_scales, int radius_prev, int radius_own, int B,
+                                    int H, int32_t* kv_cnt, int32_t* kv_idx, int32_t* order,
+                                    int32_t* done, void* stream) {
+  if (B < 1 || H < 1 || B > 65535 || H > 65535)
+    return fail(SPARVAR_ERR_INVALID_ARG, "B=%d H=%d outside [1, 65535]", B, H);
+  if (!order || !done) return fail(SPARVAR_ERR_INVALID_ARG, "order/done is NULL");
+  if (!sides || n_scales < 1 || q_scale < 0 || q_scale >= n_scales)
+    return fail(SPARVAR_ERR_INVALID_ARG, "bad schedule or q_scale");
+  const int64_t side = sides[q_scale];
+  const int64_t T = static_cast<int64_t>(B) * H * ceil_div(side * side, 128);
+  if (T > (int64_t{1} << 30)) return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
+  int G = 0;
+  int rc = attn_grid(T, &G);
+  if (rc) return rc;
+  return csla_mask_impl(sides, n_scales, q_scale, n_sink_scales, radius_prev, radius_own, 128, 128,
+                        kv_cnt, kv_idx, nullptr, stream, sparvar::TileOrderOut{order, done, B, H, G});
+}
+
+static int csla_mask_impl(const int32_t* sides, int n_scales, int q_scale, int n_sink_scales,
+                          int radius_prev, int radius_own, int block_q, int block_kv,
+                          int32_t* kv_cnt, int32_t* kv_idx, uint8_t* blk_mask, void* stream,
+                          sparvar::TileOrderOut ord) {
   sparvar::ScaleGeometry g;
   int rc = build_geometry(sides, n_scales, &g);
   if (rc) return rc;
@@ -250,7 +285,7 @@ int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int q_scale, int
   sparvar::csla_mask_kernel<<<nqb, sparvar::kMaskThreads, smem,
                               static_cast<cudaStream_t>(stream)>>>(
       g, q_scale, n_sink_scales, radius_prev, radius_own, block_q, block_kv, nkb, kv_cnt, kv_idx,
-      blk_mask);
+      blk_mask, ord);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "csla_mask_kernel launch");
   return SPARVAR_OK;

@@ -40,6 +40,8 @@ EXPORTS = {
                                        _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _i, _i, _i, _f, _vp,
                                        _vp], _i),
     "sparvar_tile_order": ([_vp, _i, _i, _i, _i64p, _i, _vp, _vp], _i),
+    "sparvar_build_csla_mask_ordered": ([_i32p, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                                         _vp], _i),
     "sparvar_block_sparse_attn_fwd_ordered": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64p,
                                                _i64p, _i64p, _i64p, _vp, _vp, _i64p, _i, _vp, _f,
                                                _vp, _vp], _i),
@@ -133,6 +135,30 @@ def sparvar_build_csla_mask(sides, q_scale, n_sink_scales, radius_prev, radius_o
                                          radius_own, block_q, block_kv, _ptr(cnt), _ptr(idx),
                                          _ptr(mask), _stream(cnt.device)), "sparvar_build_csla_mask")
     return cnt, idx, mask
+
+
+def sparvar_build_csla_mask_ordered(sides, q_scale, n_sink_scales, radius_prev, radius_own, B, H,
+                                    device="cuda", done=None, out=None):
+    """CSLA lists over 128x128 blocks and, from the same launch, the longest-first
+    tile order for a (B, H) attention call over them: (kv_cnt, kv_idx, order).
+    ``done`` is a zeroed int32 device counter the launch leaves at zero (one per
+    call site that may run concurrently); allocated here when not given."""
+    nqb, nkb = scale_blocks(sides, q_scale, 128, 128)
+    cnt = torch.empty(nqb, dtype=torch.int32, device=device)
+    idx = torch.empty(nqb, nkb, dtype=torch.int32, device=device)
+    order = out if out is not None else torch.empty(B * H * nqb, dtype=torch.int32, device=device)
+    if order.dtype != torch.int32 or order.numel() != B * H * nqb or not order.is_contiguous():
+        raise SparvarError(f"out must be a contiguous int32 tensor of {B * H * nqb}")
+    if done is None:
+        done = torch.zeros(1, dtype=torch.int32, device=device)
+    if done.dtype != torch.int32 or done.numel() != 1:
+        raise SparvarError("done must be one int32")
+    arr = (ctypes.c_int32 * len(sides))(*sides)
+    _check(lib().sparvar_build_csla_mask_ordered(arr, len(sides), q_scale, n_sink_scales, radius_prev,
+                                                 radius_own, B, H, _ptr(cnt), _ptr(idx), _ptr(order),
+                                                 _ptr(done), _stream(cnt.device)),
+           "sparvar_build_csla_mask_ordered")
+    return cnt, idx, order
 
 
 def _list_strides(kv_cnt, B, H):

@@ -106,6 +106,22 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
                             uint8_t* blk_mask, void* stream);
 
 /*
+ * sparvar_build_csla_mask at block_q = block_kv = 128 (no blk_mask) that also
+ * writes, in the same launch, the longest-first tile order of sparvar_tile_order
+ * for an attention call over B batch items and H heads sharing these lists
+ * (order: device int32 [B * H * nqb]; for launches on the current device).  The
+ * CTA that finishes last ranks the lists: done is a device int32 the caller sets
+ * to 0 once; the launch leaves it at 0.  Calls that may run at the same time
+ * need their own `done`.  Errors as for sparvar_build_csla_mask, and a NULL
+ * order or done is refused.
+ */
+SPARVAR_API int sparvar_build_csla_mask_ordered(const int32_t* sides, int n_scales, int q_scale,
+                                                int n_sink_scales, int radius_prev,
+                                                int radius_own, int B, int H, int32_t* kv_cnt,
+                                                int32_t* kv_idx, int32_t* order, int32_t* done,
+                                                void* stream);
+
+/*
  * CS4A decision: pooled softmax mass of dense attention at the sparse decision
  * scale and per-query-block selection ("Methodology in Plain English", CS4A
  * paragraph: split the dense map into query blocks, sum the attention weights

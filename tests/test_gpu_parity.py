@@ -300,6 +300,29 @@ def test_tile_order_longest_first_serpentine():
         assert all(seq[i] >= seq[i + 1] for i in range(len(seq) - 1))
 
 
+def test_csla_build_with_tile_order():
+    """The list builder's last CTA writes the same longest-first order as the order
+    call (equal list lengths at every position; ties may fall either way), the
+    lists are those of the plain builder, and the counter is back at zero, so the
+    next call can use it again."""
+    B, H = 2, 16
+    done = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for q_scale in (9, 12):
+        cnt0, idx0, _ = ops.sparvar_build_csla_mask(INF, q_scale, 5, 2, 4, 128, 128)
+        for _ in range(2):
+            cnt, idx, order = ops.sparvar_build_csla_mask_ordered(INF, q_scale, 5, 2, 4, B, H,
+                                                                  done=done)
+            torch.cuda.synchronize()
+            assert torch.equal(cnt, cnt0) and torch.equal(idx, idx0)
+            assert int(done.item()) == 0
+            nqb = cnt.numel()
+            ref = ops.sparvar_tile_order(cnt, B, H, nqb * 128)
+            c = cnt.cpu().numpy()
+            o, r = order.cpu().numpy(), ref.cpu().numpy()
+            assert sorted(o.tolist()) == list(range(B * H * nqb))
+            assert np.array_equal(c[o % nqb], c[r % nqb])
+
+
 def test_attention_in_tile_order():
     """Taking the query tiles longest first changes which CTA runs a tile and what
     comes before it (and so which softmax group takes which of its blocks, and the

@@ -214,3 +214,17 @@ def test_ordered_attention_rejects_bad_arguments(lib):
     assert "tile_order is NULL" in lib.sparvar_last_error().decode()
     assert call(16, D=96) == 2
     assert "D=96" in lib.sparvar_last_error().decode()
+
+
+def test_ordered_csla_build_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    sides = (ctypes.c_int32 * 3)(1, 2, 4)
+
+    def call(B=1, order=16, done=16, q_scale=2):
+        return lib.sparvar_build_csla_mask_ordered(sides, 3, q_scale, 1, 1, 1, B, 1, vp(16),
+                                                   vp(16), vp(order), vp(done), vp(0))
+
+    assert call(order=0) == 1 and "order/done is NULL" in lib.sparvar_last_error().decode()
+    assert call(done=0) == 1 and "order/done is NULL" in lib.sparvar_last_error().decode()
+    assert call(B=0) == 1 and "B=0" in lib.sparvar_last_error().decode()
+    assert call(q_scale=3) == 1 and "q_scale" in lib.sparvar_last_error().decode()
