@@ -31,7 +31,7 @@ from block_sparse_cross_sparvar_b200 import inputs  # noqa: E402
 WORKLOAD = dict(name="infinity2b_last_scale_64x64", sides=inputs.INFINITY_SIDES, q_scale=12,
                 B=2, H=16, D=128, n_sink_scales=5, radius_prev=2, radius_own=4, block=128)
 FLUSH_BYTES = 256 << 20
-E2E_HEADS = 4  # heads per chunk of the end-to-end pipeline
+E2E_HEADS = 2  # heads per chunk of the end-to-end pipeline
 
 
 def peaks():
