@@ -66,69 +66,107 @@ __device__ __forceinline__ void compact_bitset(const uint32_t* bits, int nkb, in
   if (lane == 0) *cnt_out = base;
 }
 
-// Order of the query tiles for the persistent attention kernel: longest lists
-// first, dealt to the kernel's G CTAs in a serpentine (round i of G tiles goes to
-// CTAs 0..G-1 when i is even and G-1..0 when i is odd), so that each CTA's total
-// work is close to the mean.  The kernel's CTA c takes the tiles at positions
-// c, c + G, c + 2G, ... of `order`.  Tile id = (b * H + h) * nqb + qb.  One CTA:
-// a histogram of the list lengths (clamped to kOrderBuckets - 1; ties in any
-// order), a scan for each length's first position, then one position per tile.
-// The counts are read through L2 (they may have been written by other CTAs of
-// the same launch).
-constexpr int kOrderBuckets = 1024;
+// Order of the query tiles for the persistent attention kernel on G CTAs, whose
+// CTA c takes the tiles at positions c, c + G, c + 2G, ... of `order` (tile id =
+// (b * H + h) * nqb + qb).  Round r is the natural tiles r*G .. r*G + G - 1 (the
+// kernel's r-th wave, so the waves keep touching the K/V of the same heads); a
+// round's tiles are ranked longest list first, then by query block, then by tile
+// id, and dealt in a serpentine: to CTAs 0..G-1 in even rounds and G-1..0 in odd
+// ones, so that each CTA's total work is close to the mean.  The counts are read
+// through L2 (they may have been written by other CTAs of the same launch).
+constexpr int kOrderMaxG = 1024;
+constexpr int kOrderSlots = 4096;  // list lengths held in shared memory at a time
+constexpr int kOrderMaxQb = 1024;
+
+__device__ __forceinline__ int clamp_len(int n, int idx_row_len) {
+  return n < 0 ? 0 : (n > idx_row_len ? idx_row_len : n);
+}
+
+// Lists per (b, h, query block): the lengths of a run of whole rounds go to shared
+// memory, then each tile's rank is the number of its round's tiles ranked before
+// it (G compares per tile).
 __device__ void order_tiles_block(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H,
                                   int nqb, int idx_row_len, int G, int32_t* order) {
-  __shared__ int hist[kOrderBuckets];
-  __shared__ int part[32];
+  __shared__ int len[kOrderSlots];
   const int T = B * H * nqb;
-  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  auto bucket = [&](int t) {
-    const int qb = t % nqb, bh = t / nqb;
-    int n = __ldcg(kv_cnt + (bh / H) * sb + (bh % H) * sh + qb);
-    n = n < 0 ? 0 : (n > idx_row_len ? idx_row_len : n);
-    return kOrderBuckets - 1 - (n < kOrderBuckets - 1 ? n : kOrderBuckets - 1);  // longest first
-  };
-  for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[bucket(t)], 1);
-  __syncthreads();
-  // exclusive scan of the histogram: each thread takes per = kOrderBuckets / blockDim.x
-  // consecutive buckets, then the threads' totals are scanned across warps
-  const int per = kOrderBuckets / blockDim.x;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int tot = 0;
-  for (int i = 0; i < per; ++i) tot += hist[threadIdx.x * per + i];
-  int x = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) part[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int v = lane < (blockDim.x >> 5) ? part[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += y;
+  const int span = (kOrderSlots / G) * G;
+  for (int c0 = 0; c0 < T; c0 += span) {
+    const int n = min(span, T - c0);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int t = c0 + i, qb = t % nqb, bh = t / nqb;
+      len[i] = clamp_len(__ldcg(kv_cnt + (bh / H) * sb + (bh % H) * sh + qb), idx_row_len);
     }
-    part[lane] = v;  // inclusive over warps
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int rs = (i / G) * G, nr = min(G, n - rs), own = i - rs;
+      const int li = len[i], qi = (c0 + i) % nqb;
+      int qu = (c0 + rs) % nqb, rank = 0;
+#pragma unroll 4
+      for (int u = 0; u < nr; ++u) {
+        const int lu = len[rs + u];
+        rank += (lu > li) | ((lu == li) & ((qu < qi) | ((qu == qi) & (u < own))));
+        qu = qu + 1 == nqb ? 0 : qu + 1;
+      }
+      const bool odd = ((c0 + rs) / G) & 1;
+      order[c0 + rs + (odd ? nr - 1 - rank : rank)] = c0 + i;
+    }
+    __syncthreads();
+  }
+}
+
+// The same order for lists shared by every (b, h) (kv_cnt[qb]): the query blocks
+// are ranked once (longest first, then by index); then one warp per round takes
+// them in that order, 32 at a time: a query block's tiles in the round (every
+// nqb-th tile) take, in tile-id order, the positions after those of the query
+// blocks ranked before it (a warp scan of the per-block counts).  nqb <= kOrderMaxQb.
+__device__ void order_tiles_shared_lists(const int32_t* kv_cnt, int B, int H, int nqb,
+                                         int idx_row_len, int G, int32_t* order) {
+  __shared__ int len_q[kOrderMaxQb];
+  __shared__ int qb_at[kOrderMaxQb];
+  for (int q = threadIdx.x; q < nqb; q += blockDim.x) len_q[q] = clamp_len(__ldcg(kv_cnt + q), idx_row_len);
+  __syncthreads();
+  for (int q = threadIdx.x; q < nqb; q += blockDim.x) {
+    const int lq = len_q[q];
+    int rank = 0;
+#pragma unroll 8
+    for (int u = 0; u < nqb; ++u) rank += (len_q[u] > lq) | ((len_q[u] == lq) & (u < q));
+    qb_at[rank] = q;
   }
   __syncthreads();
-  int start = x - tot + (w > 0 ? part[w - 1] : 0);
-  __syncthreads();
-  for (int i = 0; i < per; ++i) {
-    const int h = hist[threadIdx.x * per + i];
-    hist[threadIdx.x * per + i] = start;
-    start += h;
+  const int T = B * H * nqb, rounds = (T + G - 1) / G;
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int r = threadIdx.x >> 5; r < rounds; r += nwarps) {
+    const int r0 = r * G, nr = min(G, T - r0), r1 = r0 + nr, rm = r0 % nqb;
+    const bool odd = r & 1;
+    int p = 0;  // positions taken by the query blocks ranked before this chunk of 32
+    for (int s0 = 0; s0 < nqb; s0 += 32) {
+      int u0 = 0, c = 0;
+      if (s0 + lane < nqb) {
+        const int q = qb_at[s0 + lane];
+        u0 = r0 + (q >= rm ? q - rm : q - rm + nqb);  // the round's first tile of query block q
+        c = u0 < r1 ? (r1 - 1 - u0) / nqb + 1 : 0;
+      }
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      for (int k = 0; k < c; ++k) {
+        const int pos = p + incl - c + k;
+        order[r0 + (odd ? nr - 1 - pos : pos)] = u0 + k * nqb;
+      }
+      p += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const int pos = atomicAdd(&hist[bucket(t)], 1);  // the tile's rank, longest first
-    const int r = pos / G, j = pos % G;
-    const int in_round = min(G, T - r * G);
-    order[r * G + ((r & 1) ? in_round - 1 - j : j)] = t;
-  }
+}
+
+// The order on its own: one CTA of 1024 threads.
+__global__ void __launch_bounds__(1024)
+    tile_order_kernel(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H, int nqb,
+                      int idx_row_len, int G, int32_t* order) {
+  order_tiles_block(kv_cnt, sb, sh, B, H, nqb, idx_row_len, G, order);
 }
 
 // ---------------------------------------------------------------- CSLA
@@ -139,7 +177,7 @@ __device__ void order_tiles_block(const int32_t* kv_cnt, int64_t sb, int64_t sh,
 // the per-query windows is that rectangle).  Each key row of the rectangle is a
 // contiguous token range, which sets a contiguous range of KV-block bits.
 // With `order` set, the CTA that finishes last (counted in *done, which it sets
-// back to zero) also writes the longest-first tile order of the lists for a
+// back to zero) also writes the tile order of the lists for a
 // (B, H) launch of the attention kernel on G CTAs (the lists are shared by every
 // batch item and head).
 struct TileOrderOut {
@@ -201,7 +239,7 @@ __global__ void __launch_bounds__(kMaskThreads)
     __syncthreads();
     if (last) {
       __threadfence();
-      order_tiles_block(kv_cnt, 0, 0, ord.B, ord.H, gridDim.x, nkb, ord.G, ord.order);
+      order_tiles_shared_lists(kv_cnt, ord.B, ord.H, gridDim.x, nkb, ord.G, ord.order);
       if (threadIdx.x == 0) *ord.done = 0;
     }
   }
@@ -454,13 +492,6 @@ __global__ void validate_lists_kernel(const int32_t* kv_cnt, const int32_t* kv_i
   }
   flags = __reduce_or_sync(0xffffffffu, flags);
   if (lane == 0 && flags) atomicOr(dev_status, flags);
-}
-
-// The order on its own: one CTA of 1024 threads.
-__global__ void __launch_bounds__(1024)
-    tile_order_kernel(const int32_t* kv_cnt, int64_t sb, int64_t sh, int B, int H, int nqb,
-                      int idx_row_len, int G, int32_t* order) {
-  order_tiles_block(kv_cnt, sb, sh, B, H, nqb, idx_row_len, G, order);
 }
 
 }  // namespace sparvar

@@ -253,11 +253,15 @@ int sparvar_build_csla_mask_ordered(const int32_t* sides, int n_scales, int q_sc
   if (!sides || n_scales < 1 || q_scale < 0 || q_scale >= n_scales)
     return fail(SPARVAR_ERR_INVALID_ARG, "bad schedule or q_scale");
   const int64_t side = sides[q_scale];
-  const int64_t T = static_cast<int64_t>(B) * H * ceil_div(side * side, 128);
+  const int64_t nqb = ceil_div(side * side, 128);
+  if (nqb > sparvar::kOrderMaxQb)
+    return fail(SPARVAR_ERR_UNSUPPORTED, "more than %d query blocks", sparvar::kOrderMaxQb);
+  const int64_t T = static_cast<int64_t>(B) * H * nqb;
   if (T > (int64_t{1} << 30)) return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
   int G = 0;
   int rc = attn_grid(T, &G);
   if (rc) return rc;
+  if (G > sparvar::kOrderMaxG) return fail(SPARVAR_ERR_UNSUPPORTED, "more than %d SMs", G);
   return csla_mask_impl(sides, n_scales, q_scale, n_sink_scales, radius_prev, radius_own, 128, 128,
                         kv_cnt, kv_idx, nullptr, stream, sparvar::TileOrderOut{order, done, B, H, G});
 }
@@ -281,7 +285,8 @@ static int csla_mask_impl(const int32_t* sides, int n_scales, int q_scale, int n
   const int nqb = static_cast<int>(ceil_div(nq, block_q));
   const int nkb = static_cast<int>(ceil_div(g.off[q_scale + 1], block_kv));
   const size_t smem = static_cast<size_t>((nkb + 31) / 32) * 4;
-  if (smem > 48 * 1024) return fail(SPARVAR_ERR_UNSUPPORTED, "too many KV blocks (%d)", nkb);
+  // the kernel's static shared memory (the order's 8 KB) and the bitset share 48 KB
+  if (smem > 40 * 1024) return fail(SPARVAR_ERR_UNSUPPORTED, "too many KV blocks (%d)", nkb);
   sparvar::csla_mask_kernel<<<nqb, sparvar::kMaskThreads, smem,
                               static_cast<cudaStream_t>(stream)>>>(
       g, q_scale, n_sink_scales, radius_prev, radius_own, block_q, block_kv, nkb, kv_cnt, kv_idx,
@@ -613,7 +618,8 @@ int sparvar_tile_order(const int32_t* kv_cnt, int B, int H, int Lq,
   if (T > (int64_t{1} << 30)) return fail(SPARVAR_ERR_UNSUPPORTED, "more than 2^30 query tiles");
   int G = 0, rc;
   if ((rc = attn_grid(T, &G))) return rc;
-  sparvar::tile_order_kernel<<<1, sparvar::kOrderBuckets, 0, static_cast<cudaStream_t>(stream)>>>(
+  if (G > sparvar::kOrderMaxG) return fail(SPARVAR_ERR_UNSUPPORTED, "more than %d SMs", G);
+  sparvar::tile_order_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
       kv_cnt, list_strides[0], list_strides[1], B, H, static_cast<int>(nqb), idx_row_len, G, order);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile_order_kernel launch");

@@ -107,7 +107,7 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
 
 /*
  * sparvar_build_csla_mask at block_q = block_kv = 128 (no blk_mask) that also
- * writes, in the same launch, the longest-first tile order of sparvar_tile_order
+ * writes, in the same launch, the tile order of sparvar_tile_order
  * for an attention call over B batch items and H heads sharing these lists
  * (order: device int32 [B * H * nqb]; for launches on the current device).  The
  * CTA that finishes last ranks the lists: done is a device int32 the caller sets
@@ -283,17 +283,20 @@ SPARVAR_API int sparvar_block_sparse_attn_fwd(const void* q, const void* k, cons
                                   void* stream);
 
 /*
- * Longest lists first (a scheduling aid for the persistent attention kernel; the
- * pages fix no tile order): writes into order[T], T = B * H * ceil(Lq / 128), the
- * tile ids (b * H + h) * nqb + qb sorted by list length, longest first, then dealt
- * to the kernel's G = min(T, SMs of the current device) CTAs in a serpentine
- * (round i of G tiles to CTAs 0..G-1 for even i, G-1..0 for odd i), so that each
- * CTA's total list length is close to the mean.  Lengths above 1022 count as 1023;
- * ties are taken in any order.  kv_cnt, list_strides and idx_row_len as for
- * sparvar_block_sparse_attn_fwd with 128x128 blocks; order is device int32 owned
- * by the caller.  One launch of one CTA on `stream`; the order depends on the
- * device's SM count, so it is for launches on that device.  Errors: a bad shape
- * or pointer is refused before anything is enqueued.
+ * Longest lists first, wave by wave (a scheduling aid for the persistent
+ * attention kernel; the pages fix no tile order): writes into order[T], T = B * H *
+ * ceil(Lq / 128), the tile ids (b * H + h) * nqb + qb for the kernel's
+ * G = min(T, SMs of the current device) CTAs, CTA c taking positions c, c + G, ...
+ * Round r holds the natural tiles r*G .. r*G + G - 1 (so that each wave of the
+ * kernel touches the same heads' K/V as in natural order), ranked longest list
+ * first, then by query block qb, then by tile id, and dealt to CTAs 0..G-1 for
+ * even r and G-1..0 for odd
+ * r, so that each CTA's total work is close to the mean.  kv_cnt, list_strides
+ * and idx_row_len as for sparvar_block_sparse_attn_fwd with 128x128 blocks;
+ * order is device int32 owned by the caller.  One launch of one CTA on `stream`
+ * (G compares per tile); the order depends on the device's SM count, so it is for
+ * launches on that device.  Errors: a bad shape or pointer is refused before
+ * anything is enqueued.
  */
 SPARVAR_API int sparvar_tile_order(const int32_t* kv_cnt, int B, int H, int Lq,
                                    const int64_t* list_strides, int idx_row_len, int32_t* order,

@@ -277,9 +277,9 @@ def test_attention_persistent_short_and_empty_lists(D):
 
 
 def test_tile_order_longest_first_serpentine():
-    """The order is a permutation of the tiles; round r of G positions holds the r-th
-    G longest lists (longest first over the whole order), dealt to CTAs 0..G-1 for
-    even r and G-1..0 for odd r."""
+    """The order is a permutation of the tiles; round r of G positions holds the
+    natural tiles r*G .. r*G + G - 1, longest list first, then by query block, then
+    by tile id, dealt to CTAs 0..G-1 for even r and G-1..0 for odd r."""
     rng = np.random.default_rng(5)
     B, H, nqb = 2, 16, 40
     lens = rng.integers(0, 30, size=(B, H, nqb)).astype(np.int32)
@@ -289,25 +289,20 @@ def test_tile_order_longest_first_serpentine():
     G = min(T, torch.cuda.get_device_properties(0).multi_processor_count)
     assert sorted(order.tolist()) == list(range(T))
     flat = lens.reshape(-1)
-    ranked = np.sort(flat)[::-1]
     for r in range(-(-T // G)):
         pos = order[r * G:(r + 1) * G]
-        got = flat[pos]
-        # this round holds exactly the next lengths of the ranking
-        assert sorted(got.tolist()) == sorted(ranked[r * G:(r + 1) * G].tolist())
-        # and deals them longest first in its direction
-        seq = got if r % 2 == 0 else got[::-1]
-        assert all(seq[i] >= seq[i + 1] for i in range(len(seq) - 1))
+        tiles = np.arange(r * G, min(T, (r + 1) * G))
+        want = sorted(tiles.tolist(), key=lambda t: (-flat[t], t % nqb, t))
+        dealt = pos if r % 2 == 0 else pos[::-1]
+        assert dealt.tolist() == want
 
 
 def test_csla_build_with_tile_order():
-    """The list builder's last CTA writes the same longest-first order as the order
-    call (equal list lengths at every position; ties may fall either way), the
+    """The list builder's last CTA writes the same order as the order call, the
     lists are those of the plain builder, and the counter is back at zero, so the
     next call can use it again."""
-    B, H = 2, 16
     done = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for q_scale in (9, 12):
+    for q_scale, B, H in ((9, 2, 16), (12, 2, 16), (12, 1, 5), (11, 3, 25)):
         cnt0, idx0, _ = ops.sparvar_build_csla_mask(INF, q_scale, 5, 2, 4, 128, 128)
         for _ in range(2):
             cnt, idx, order = ops.sparvar_build_csla_mask_ordered(INF, q_scale, 5, 2, 4, B, H,
@@ -317,10 +312,7 @@ def test_csla_build_with_tile_order():
             assert int(done.item()) == 0
             nqb = cnt.numel()
             ref = ops.sparvar_tile_order(cnt, B, H, nqb * 128)
-            c = cnt.cpu().numpy()
-            o, r = order.cpu().numpy(), ref.cpu().numpy()
-            assert sorted(o.tolist()) == list(range(B * H * nqb))
-            assert np.array_equal(c[o % nqb], c[r % nqb])
+            assert torch.equal(order, ref)
 
 
 def test_attention_in_tile_order():
@@ -401,17 +393,23 @@ def test_attention_bad_list_entries_flagged_not_trapped():
 
 def test_attention_full_size_sampled_rows():
     """Infinity-2B last scale (B2 H16, 4096 x 10521, D128) in the bench's launch
-    configuration; sampled rows against the oracle evaluated row by row."""
+    configuration (the list builder's tile order); sampled rows against the oracle
+    evaluated row by row, and the natural tile order within rounding."""
     d = inputs.make_qkv(0, 2, 16, INF, 128, 5)
     off = d["offsets"]
     q_bits = d["q"][:, :, off[12]:off[13]]
     q, k, v = _dev(q_bits), _dev(d["k"]), _dev(d["v"])
-    cnt, idx, _ = ops.sparvar_build_csla_mask(INF, 12, 5, 2, 4, 128, 128)
+    done = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cnt, idx, order = ops.sparvar_build_csla_mask_ordered(INF, 12, 5, 2, 4, 2, 16, done=done)
     st = _status()
-    o, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True, dev_status=st)
+    o, lse = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, return_lse=True, dev_status=st,
+                                               tile_order=order)
+    o_nat = ops.sparvar_block_sparse_attn_fwd(q, k, v, cnt, idx, dev_status=st)
     torch.cuda.synchronize()
     assert st.item() == 0
+    assert (o.float() - o_nat.float()).abs().max().item() <= 1e-2
     ocnt, oidx, blk = orc.build_csla_mask(INF, 12, 5, 2, 4, 128, 128)
+    assert np.array_equal(cnt.cpu().numpy(), ocnt) and np.array_equal(idx.cpu().numpy(), oidx)
     rng = np.random.default_rng(0)
     errs = []
     for b, h in [(0, 0), (1, 15), (0, 7), (1, 3)]:
