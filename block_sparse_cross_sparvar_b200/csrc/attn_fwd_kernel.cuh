@@ -23,11 +23,14 @@
 // issuer 0 once the previous tile's MMAs have all completed.  Block j's group
 // is PV_j followed by S_{j+3} into the buffer PV_j has just read (one issuer's
 // MMAs run in issue order); issuer J mod 2 runs it, so while one issuer waits
-// on a barrier the other keeps the tensor core's short queue filled.  Each
-// group commits once on rel[G mod 16] (G numbers the groups of the sequence in
-// order), which frees its ring slots; the producer records, per slot, the group
-// that must release it.  Release barriers outnumber ring slots, so no waiter can
-// fall two phases behind a barrier.
+// on a barrier the other keeps the tensor core's short queue filled.  The issuer
+// waits for P_J and V_j, issues the PV MMAs and commits on rel_v[G mod 16] (G
+// numbers the groups of the sequence in order), which frees V_j's slot; only then
+// does it wait for K_{j+3}, whose load is the one most often late, and after the
+// score MMAs it commits on rel[G mod 16], which frees K_{j+3}'s slot.  The
+// producer records, per slot, the group that must release it and whether it held
+// a V block.  Release barriers outnumber ring slots, so no waiter can fall two
+// phases behind a barrier.
 //
 // Softmax.  Both groups add into one O, so they share a per-row reference max
 // m (log2 units) in shared memory, reset at each tile.  Block J is computed
@@ -119,6 +122,7 @@ struct __align__(8) Bars {
   uint64_t epi[2];                // epilogue of non-empty tile k done: [k & 1], phase k >> 1
   uint64_t full[kMaxSlots];       // ring slot loaded (TMA transaction count)
   uint64_t rel[kRel];             // MMA group G done: [G % kRel], phase G / kRel
+  uint64_t rel_v[kRel];           // the PV MMAs of group G done (its V slot free): same indexing
   uint64_t s_full[3], p_full[3];  // block J: [J % 3], phase J / 3
   uint64_t o_done[2];             // every PV of non-empty tile k done: [k & 1], phase k >> 1
   uint64_t drain;
@@ -316,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_sh;
   __shared__ float m_sh[kTile];      // shared reference max per row
   __shared__ int relg_sh[kMaxSlots];  // producer: group that frees each ring slot (-1: unused)
+  __shared__ int relv_sh[kMaxSlots];  // producer: the slot holds a V block (freed by rel_v)
 
   const uint32_t smem_base = (smem_addr(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_addr(smem_raw));
@@ -334,7 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.epi[i], 1);
     }
     for (int s = 0; s < NS; ++s) mbar_init(&bars.full[s], 1);
-    for (int i = 0; i < kRel; ++i) mbar_init(&bars.rel[i], 1);
+    for (int i = 0; i < kRel; ++i) {
+      mbar_init(&bars.rel[i], 1);
+      mbar_init(&bars.rel_v[i], 1);
+    }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 128);
@@ -344,7 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (threadIdx.x < kTile) m_sh[threadIdx.x] = -INFINITY;
-  if (threadIdx.x < kMaxSlots) relg_sh[threadIdx.x] = -1;
+  if (threadIdx.x < kMaxSlots) {
+    relg_sh[threadIdx.x] = -1;
+    relv_sh[threadIdx.x] = 0;
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(&tmem_base_sh, kTmemCols);
     tmem_relinquish();
@@ -376,11 +387,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto produce = [&](const CUtensorMap* tm, int kb, int grp, const TileCoord& tc) {
         const int s = w % NS;
         const int prev = relg_sh[s];
-        if (prev >= 0 && !wait_group(bars.rel, prev, abort_flag, dev_status)) {
+        if (prev >= 0 &&
+            !wait_group(relv_sh[s] ? bars.rel_v : bars.rel, prev, abort_flag, dev_status)) {
           ok = false;
           return;
         }
         relg_sh[s] = grp;
+        relv_sh[s] = tm == &tm_v;
         kb = kb < 0 ? -1 : (kb > tc.nkb ? tc.nkb : kb);
         mbar_arrive_expect_tx(&bars.full[s], L::kTileBytes);
 #pragma unroll
@@ -485,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bars.s_full[(c.J0 + jj) % 3]);
           }
           if (!ok) break;
+          mma_commit(&bars.rel_v[group_of_prologue(c) % kRel]);  // (no PV: keeps the phases)
           mma_commit(&bars.rel[group_of_prologue(c) % kRel]);
         }
         for (int j = ((c.J0 & 1) == me) ? 0 : 1; j < c.n && ok; j += 2) {
@@ -494,10 +508,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool more = has_k_after(c, j);
           const bool feed = more && j >= nk;  // S of the next tile's block j - nk
           wait_pos(pv);
-          if (more) wait_pos(pv + 1);
-          if (feed)
-            ok = ok && mbar_wait(&bars.q_full[(c.k + 1) & 1], ((c.k + 1) >> 1) & 1, abort_flag,
-                                 dev_status, 0x2, kWaitNs);
           if (!ok) break;
           const uint64_t dvs = dv + static_cast<uint64_t>((pv % NS) * kBufStep);
           const uint32_t a_col = tmem + (J % 3) * 128;
@@ -508,7 +518,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                    idesc_pv, 1u);
           // this issuer's last PV of the tile: O is final once both issuers' are done
           if (j + 2 >= c.n) mma_commit(&bars.o_done[c.k & 1]);
+          mma_commit(&bars.rel_v[group_of_block(c, j) % kRel]);
+          // the score MMAs' operands are waited for only now, behind the PV MMAs
+          if (more) wait_pos(pv + 1);
+          if (feed)
+            ok = ok && mbar_wait(&bars.q_full[(c.k + 1) & 1], ((c.k + 1) >> 1) & 1, abort_flag,
+                                 dev_status, 0x2, kWaitNs);
+          if (!ok) break;
           if (more) {
+            tc_fence_after();
             // buffer J mod 3 is free once PV_J has read P_J (this issuer's MMAs run in order)
             issue_s(J + 3, feed ? c.k + 1 : c.k, pv + 1);
             mma_commit(&bars.s_full[J % 3]);
@@ -679,11 +697,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O holds non-zero values only once an earlier block of the tile had a finite reference
         const bool o_live = raise && m_fin != -INFINITY;
         if (__any_sync(0xffffffffu, o_live)) {
-          // every earlier PV of the tile is complete once the latest group of each
-          // issuer (blocks j-1 and j-2) has completed
-          if (!warp_wait_group(bars.rel, group_of_block(c, j - 1), abort_flag, dev_status) ||
+          // every earlier PV of the tile is complete once the PV MMAs of the latest
+          // group of each issuer (blocks j-1 and j-2) have completed
+          if (!warp_wait_group(bars.rel_v, group_of_block(c, j - 1), abort_flag, dev_status) ||
               (j >= 2 &&
-               !warp_wait_group(bars.rel, group_of_block(c, j - 2), abort_flag, dev_status))) {
+               !warp_wait_group(bars.rel_v, group_of_block(c, j - 2), abort_flag, dev_status))) {
             good = false;
             break;
           }

@@ -17,12 +17,15 @@ the score MMA of block J + 3, also across a tile boundary when the tile has at
 least three blocks (it then feeds the next tile: the next tile's Q and first
 K blocks are loaded in its ring stream); a tile whose predecessor is shorter
 starts with a prologue group issued by issuer 0 after the predecessor's MMAs;
-groups commit on rel[G mod 16] and each issuer signs a per-tile o_done after
-its last PV of the tile, which the epilogue waits for; an issuer waits for its
-block's P before the block's V and K ring slots (a slot may be two loads
-behind before then); the producer waits for the group that last used a ring
-slot; Q buffers alternate between non-empty tiles and come back after each
-tile's epilogue.  Known-bad
+groups commit on rel[G mod 16], and on rel_v[G mod 16] once their PV MMAs are
+issued (a prologue group, which has none, commits it with rel); each issuer
+signs a per-tile o_done after its last PV of the tile, which the epilogue waits
+for; an issuer waits for its block's P and V slot, issues the PV MMAs, and only
+then waits for the K slot (and the next Q when it feeds); the producer waits,
+for a ring slot, on rel_v of the group that last read a V block from it and on
+rel of the group that last read a K block; an O rescale waits on rel_v of the
+latest group of each issuer; Q buffers alternate between non-empty tiles and
+come back after each tile's epilogue.  Known-bad
 variants (waiting for P of the next block inside the current MMA group; fewer
 release barriers than the protocol needs; waiting for ring slots before P) are
 checked to fail, so the checker is not vacuous.
@@ -78,6 +81,7 @@ class Model:
             self.bars[f"full{i}"] = Bar()
         for i in range(n_rel):
             self.bars[f"rel{i}"] = Bar()
+            self.bars[f"rel_v{i}"] = Bar()
         for i in range(3):
             self.bars[f"s_full{i}"] = Bar()
             self.bars[f"p_full{i}"] = Bar()
@@ -122,6 +126,9 @@ class Model:
     def rel(self, g):
         return ("wait", f"rel{g % self.n_rel}", g // self.n_rel)
 
+    def rel_v(self, g):
+        return ("wait", f"rel_v{g % self.n_rel}", g // self.n_rel)
+
     def full(self, p):
         return ("wait", f"full{p % self.ns}", p // self.ns)
 
@@ -135,8 +142,9 @@ class Model:
                 continue
             s = w % self.ns
             if owner[s] is not None:
-                yield self.rel(owner[s])
-            owner[s] = g
+                og, ov = owner[s]
+                yield self.rel_v(og) if ov else self.rel(og)
+            owner[s] = (g, kind == "V")
             yield ("tma", f"full{s}")
             w += 1
         yield ("end",)
@@ -151,6 +159,7 @@ class Model:
             yield self.full(self.pos[("K", d["J0"] + jj)])
             yield ("issue",)
             yield ("commit", f"s_full{(d['J0'] + jj) % 3}")
+        yield ("commit", f"rel_v{d['Gpro'] % self.n_rel}")
         yield ("commit", f"rel{d['Gpro'] % self.n_rel}")
 
     def issuer(self, me):
@@ -163,19 +172,22 @@ class Model:
                 if X % 2 != me:
                     continue
                 x = self.k_after(d, j)
-                if not self.bad_slots_first:
-                    yield ("wait", f"p_full{X % 3}", X // 3)
-                yield self.full(self.pos[("V", X)])
-                if x is not None:
-                    yield self.full(self.pos[("K", x)])
-                    if j + 3 >= d["n"]:
-                        yield ("wait", f"q_full{d['next']['k'] % 2}", d["next"]["k"] // 2)
                 if self.bad_slots_first:
-                    yield ("wait", f"p_full{X % 3}", X // 3)
+                    yield self.full(self.pos[("V", X)])
+                    if x is not None:
+                        yield self.full(self.pos[("K", x)])
+                yield ("wait", f"p_full{X % 3}", X // 3)
+                if not self.bad_slots_first:
+                    yield self.full(self.pos[("V", X)])
                 yield ("issue",)
                 if j + 2 >= d["n"]:  # this issuer's last PV of the tile
                     yield ("commit", f"o_done{d['k'] % 2}")
+                yield ("commit", f"rel_v{(d['G0'] + j) % self.n_rel}")
                 if x is not None:
+                    if not self.bad_slots_first:
+                        yield self.full(self.pos[("K", x)])
+                    if j + 3 >= d["n"]:
+                        yield ("wait", f"q_full{d['next']['k'] % 2}", d["next"]["k"] // 2)
                     yield ("issue",)
                     yield ("commit", f"s_full{X % 3}")
                 yield ("commit", f"rel{(d['G0'] + j) % self.n_rel}")
@@ -187,7 +199,8 @@ class Model:
         yield ("end",)
 
     def issuer_bad(self, me):
-        """Issuer 0 alone, waiting for P_{J+1} inside group J (deadlocks on a raise)."""
+        """Issuer 0 alone, waiting for P_{J+1} inside group J, before the group's
+        commits (deadlocks on a raise)."""
         if me == 1:
             for d in self.desc:
                 yield ("commit", f"o_done{d['k'] % 2}")
@@ -215,6 +228,7 @@ class Model:
                         yield ("wait", f"q_full{d['next']['k'] % 2}", d["next"]["k"] // 2)
                     yield ("issue",)
                     yield ("commit", f"s_full{X % 3}")
+                yield ("commit", f"rel_v{(d['G0'] + j) % self.n_rel}")
                 yield ("commit", f"rel{(d['G0'] + j) % self.n_rel}")
             prev = d
         yield ("commit", "drain")
@@ -231,10 +245,10 @@ class Model:
                 if X > 0:
                     yield ("wait", f"p_full{(X - 1) % 3}", (X - 1) // 3)
                 if j > 0 and self.rng.random() < self.p_raise:
-                    # O rescale: the latest group of each issuer must have completed
-                    yield self.rel(d["G0"] + j - 1)
+                    # O rescale: the PVs of the latest group of each issuer must have completed
+                    yield self.rel_v(d["G0"] + j - 1)
                     if j > 1:
-                        yield self.rel(d["G0"] + j - 2)
+                        yield self.rel_v(d["G0"] + j - 2)
                 yield ("arrive", f"p_full{X % 3}")
             # epilogue: every PV of the tile has completed (o_done), then a named
             # barrier of both groups, then the Q buffer goes back to the producer
