@@ -31,7 +31,30 @@ from block_sparse_cross_sparvar_b200 import inputs  # noqa: E402
 WORKLOAD = dict(name="infinity2b_last_scale_64x64", sides=inputs.INFINITY_SIDES, q_scale=12,
                 B=2, H=16, D=128, n_sink_scales=5, radius_prev=2, radius_own=4, block=128)
 FLUSH_BYTES = 256 << 20
-E2E_HEADS = 2  # heads per chunk of the end-to-end pipeline
+def e2e_chunks(B, H):
+    """(b, h0, h1) head ranges of the end-to-end pipeline, in order.  Every copy
+    costs about 4 us on top of its bytes, so the chunks are as large as a batch
+    item allows, except towards the end, where they halve down to one head: only
+    the last chunk's compute and copy back are not hidden behind input copies."""
+    sizes, left = [], B * H
+    tail = 1
+    while left > 0:
+        take = min(tail, left)
+        sizes.append(take)
+        left -= take
+        if len(sizes) >= 2:
+            tail *= 2
+    sizes.reverse()  # large first, then 8, 4, 2, 1, 1 heads
+    chunks, b_, h0 = [], 0, 0
+    for n in sizes:
+        while n > 0:  # a chunk does not span two batch items
+            take = min(n, H - h0)
+            chunks.append((b_, h0, h0 + take))
+            n -= take
+            h0 += take
+            if h0 == H:
+                b_, h0 = b_ + 1, 0
+    return chunks
 
 
 def peaks():
@@ -344,7 +367,7 @@ def main():
     # chunk c + 1 runs while chunk c is computed and chunk c - 1 is copied back, so
     # the step approaches the time of the input copy alone.
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    chunks = [(b_, h0) for b_ in range(B) for h0 in range(0, H, E2E_HEADS)]
+    chunks = e2e_chunks(B, H)
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     s_cmp = torch.cuda.current_stream(dev)
     e2e_ms, copy_ms = [], []
@@ -353,8 +376,8 @@ def main():
         cnt_e, idx_e, _ = ops.sparvar_build_csla_mask(sides, k, wl["n_sink_scales"], wl["radius_prev"],
                                                       wl["radius_own"], bq, bq, device=dev)
         done_in, done_cmp = [], []
-        for b_, h0 in chunks:
-            sl = (slice(b_, b_ + 1), slice(h0, h0 + E2E_HEADS))
+        for b_, h0, h1 in chunks:
+            sl = (slice(b_, b_ + 1), slice(h0, h1))
             with torch.cuda.stream(s_in):
                 q[sl].copy_(hq[sl], non_blocking=True)
                 kk[sl].copy_(hk[sl], non_blocking=True)
@@ -362,16 +385,16 @@ def main():
                 ev = torch.cuda.Event()
                 ev.record(s_in)
                 done_in.append(ev)
-        for (b_, h0), ev in zip(chunks, done_in):
-            sl = (slice(b_, b_ + 1), slice(h0, h0 + E2E_HEADS))
+        for (b_, h0, h1), ev in zip(chunks, done_in):
+            sl = (slice(b_, b_ + 1), slice(h0, h1))
             s_cmp.wait_event(ev)
             ops.sparvar_block_sparse_attn_fwd(q[sl], kk[sl], vv[sl], cnt_e, idx_e, bq, bq, out=o[sl],
                                               dev_status=status)
             evc = torch.cuda.Event()
             evc.record(s_cmp)
             done_cmp.append(evc)
-        for (b_, h0), evc in zip(chunks, done_cmp):
-            sl = (slice(b_, b_ + 1), slice(h0, h0 + E2E_HEADS))
+        for (b_, h0, h1), evc in zip(chunks, done_cmp):
+            sl = (slice(b_, b_ + 1), slice(h0, h1))
             s_out.wait_event(evc)
             with torch.cuda.stream(s_out):
                 ho[sl].copy_(o[sl], non_blocking=True)
@@ -434,8 +457,9 @@ def main():
                                          "null when the source changed since the capture"},
             "e2e": {"value": total_flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": t_e2e, "input_copy_alone_ms": float(np.median(copy_ms)),
-                    "pipeline": f"{len(chunks)} chunks of {E2E_HEADS} heads: copy in, compute and "
-                                "copy out on three streams",
+                    "pipeline": f"{len(chunks)} chunks of "
+                                f"{'/'.join(str(h1 - h0) for _, h0, h1 in chunks)} heads: copy in, "
+                                "compute and copy out on three streams",
                     "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                     "d2h_bytes_per_step": int(ho.numel() * 2)},
             "gpu_launches": 2 * args.steps,
