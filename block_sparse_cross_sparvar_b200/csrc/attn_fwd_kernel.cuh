@@ -581,13 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // [i << mask_shift, (i + 1) << mask_shift) of the tile
         uint32_t keep = 0xffu;
         bool fine = false;
-        if (args.tile_mask) {
-          const int fg = kTile >> args.mask_shift;
-          const uint32_t full = (1u << fg) - 1u;
-          const uint64_t mk = __ldg(args.tile_mask + (c.list - args.prob[pi].kv_idx) + j);
-          keep = static_cast<uint32_t>(mk >> ((row >> args.mask_shift) * fg)) & full;
-          fine = __any_sync(0xffffffffu, keep != full);
-          keep |= ~full;
+        if constexpr (!ORD) {  // (launches in a given tile order take no tile masks)
+          if (args.tile_mask) {
+            const int fg = kTile >> args.mask_shift;
+            const uint32_t full = (1u << fg) - 1u;
+            const uint64_t mk = __ldg(args.tile_mask + (c.list - args.prob[pi].kv_idx) + j);
+            keep = static_cast<uint32_t>(mk >> ((row >> args.mask_shift) * fg)) & full;
+            fine = __any_sync(0xffffffffu, keep != full);
+            keep |= ~full;
+          }
         }
         // with the CSLA token mask on, bit c of km keeps column c of this row
         uint32_t km[4] = {~0u, ~0u, ~0u, ~0u};
@@ -599,6 +601,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             csla_row_mask(args.tok, gq / sk, gq % sk, kb * kTile, kb * kTile + valid, km);
           fine = true;
         }
+        // columns at or past the prefix end (the same for every row): -inf in TMEM
+        // before S is read, with whole-warp stores (the multi-problem and token-mask
+        // instantiations mask them in registers, which spills less there)
+        constexpr bool kTmemMask = !MULTI && !TOK;
+        if constexpr (kTmemMask) {
+         if (valid < kTile) {
+          const uint32_t ninf = __float_as_uint(-INFINITY);
+          const int v8 = (valid + 7) & ~7;
+          for (int col = valid; col < v8; ++col) tmem_st1(s_addr + col, ninf);
+          for (int col = v8; col < kTile; col += 8) tmem_st8_fill(s_addr + col, ninf);
+          tmem_wait_st();
+         }
+        }
         auto dropped = [&](int col) {
           return col >= valid || !((keep >> (col >> args.mask_shift)) & 1u) ||
                  !((km[col >> 5] >> (col & 31)) & 1u);
@@ -609,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           uint32_t sr[kTile];
           tmem_ld128_wait(s_addr, sr);
-          if (valid < kTile || fine) {
+          if ((!kTmemMask && valid < kTile) || fine) {
 #pragma unroll
             for (int k = 0; k < kTile; ++k)
               if (dropped(k)) sr[k] = __float_as_uint(-INFINITY);
@@ -662,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(s_addr + cc * 16, pk);
         };
         auto mask_chunk = [&](uint32_t(&cur)[32], int cc) {
-          if (valid < kTile || fine) {
+          if ((!kTmemMask && valid < kTile) || fine) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
               if (dropped(cc * 32 + k)) cur[k] = __float_as_uint(-INFINITY);
