@@ -305,7 +305,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // TOK: apply the CSLA token mask (args.tok) inside the kept tiles.  MULTI: the
 // launch holds several problems (args.prob), one output map each.
-template <int D, bool TOK, bool MULTI, bool ORD = false>
+template <int D, bool TOK, bool MULTI, bool ORD = false, bool FINE = true>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -581,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // [i << mask_shift, (i + 1) << mask_shift) of the tile
         uint32_t keep = 0xffu;
         bool fine = false;
-        if constexpr (!ORD) {  // (launches in a given tile order take no tile masks)
+        if constexpr (FINE) {  // (instantiated without it for launches with no tile masks)
           if (args.tile_mask) {
             const int fg = kTile >> args.mask_shift;
             const uint32_t full = (1u << fg) - 1u;
@@ -606,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // instantiations mask them in registers, which spills less there)
         constexpr bool kTmemMask = !MULTI && !TOK;
         if constexpr (kTmemMask) {
-         if (valid < kTile) {
+         if (__builtin_expect(valid < kTile, 0)) {
           const uint32_t ninf = __float_as_uint(-INFINITY);
           const int v8 = (valid + 7) & ~7;
           for (int col = valid; col < v8; ++col) tmem_st1(s_addr + col, ninf);
@@ -711,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_blk = raise ? bm : m_fin;  // reference of block J from now on
         // O holds non-zero values only once an earlier block of the tile had a finite reference
         const bool o_live = raise && m_fin != -INFINITY;
-        if (__any_sync(0xffffffffu, o_live)) {
+        if (__builtin_expect(__any_sync(0xffffffffu, o_live), 0)) {  // rare: laid out of line
           // every earlier PV of the tile is complete once the PV MMAs of the latest
           // group of each issuer (blocks j-1 and j-2) have completed
           if (!warp_wait_group(bars.rel_v, group_of_block(c, j - 1), abort_flag, dev_status) ||
@@ -732,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool fix_p = (m_use != m_blk) && m_use != -INFINITY;
-        if (__any_sync(0xffffffffu, fix_p)) {
+        if (__builtin_expect(__any_sync(0xffffffffu, fix_p), 0)) {
           // the shared reference moved while P_J was computed: rescale P_J to m_blk
           tmem_wait_st();
           const float beta = fix_p ? ex2_approx(m_use - m_blk) : 1.f;

@@ -142,11 +142,11 @@ int launch_decide_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const spa
   return SPARVAR_OK;
 }
 
-template <int D, bool TOK, bool MULTI, bool ORD = false>
+template <int D, bool TOK, bool MULTI, bool ORD = false, bool FINE = true>
 int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const sparvar::fwd::OutMaps& to, const sparvar::fwd::Args& a,
                       cudaStream_t stream) {
-  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI, ORD>;
+  auto kern = sparvar::fwd::attn_fwd_kernel<D, TOK, MULTI, ORD, FINE>;
   const uint32_t smem = sparvar::fwd::Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -527,10 +527,17 @@ static int attn_fwd_launch(const FwdLaunch& L, void* stream) {
     if (L.D == 128) return launch_fwd_kernel<128, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
     return launch_fwd_kernel<64, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
   }
+  // launches without tile masks (every launch in a given order) run instantiations
+  // compiled without the fine-mask code
   if (L.a.tile_order) {
     if (L.D == 128)
-      return launch_fwd_kernel<128, false, false, true>(L.tq, L.tk, L.tv, L.to, L.a, st);
-    return launch_fwd_kernel<64, false, false, true>(L.tq, L.tk, L.tv, L.to, L.a, st);
+      return launch_fwd_kernel<128, false, false, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+    return launch_fwd_kernel<64, false, false, true, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+  }
+  if (!L.a.tile_mask) {
+    if (L.D == 128)
+      return launch_fwd_kernel<128, false, false, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
+    return launch_fwd_kernel<64, false, false, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
   }
   if (L.D == 128) return launch_fwd_kernel<128, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
   return launch_fwd_kernel<64, false, false>(L.tq, L.tk, L.tv, L.to, L.a, st);
