@@ -67,7 +67,7 @@ def peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-ATTN_KERNEL = "attn_fwd_kernel<128, TOK=false, MULTI=false, ORD=true>"
+ATTN_KERNEL = "attn_fwd_kernel<128, TOK=false, MULTI=false, ORD=true, FINE=false>"
 
 
 def profiled_traffic():
