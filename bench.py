@@ -451,7 +451,9 @@ def main():
             "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL,
                          "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16"],
-                         "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']}",
+                         "frac_of_sustained": achieved / pk["bf16_sustained"],
+                         "peak_note": f"{pk['source']} bf16 dense burst; sustained {pk['bf16_sustained']} "
+                                      f"(the timed steps follow a {args.soak_s:g} s soak under the power cap)",
                          "traffic": profiled_traffic(),
                          "traffic_note": "ncu dram bytes read+write per launch of this kernel source; "
                                          "null when the source changed since the capture"},
