@@ -736,8 +736,9 @@ int sparvar_block_sparse_attn_fwd_multi(
       return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_fwd_kernel<128, false, true>(tq, tk, tv, to, a, st);
-  return launch_fwd_kernel<64, false, true>(tq, tk, tv, to, a, st);
+  // (multi-problem launches take no tile masks)
+  if (D == 128) return launch_fwd_kernel<128, false, true, false, false>(tq, tk, tv, to, a, st);
+  return launch_fwd_kernel<64, false, true, false, false>(tq, tk, tv, to, a, st);
 }
 
 int sparvar_csla_token_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
