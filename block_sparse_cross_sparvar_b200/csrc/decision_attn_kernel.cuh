@@ -520,24 +520,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        // this row's keep mask over the block's 128 columns: the keys of the prefix
-        uint32_t km[4] = {~0u, ~0u, ~0u, ~0u};
-        if ((kb + 1) * kTile > p_lkv) {
+        // the columns past the prefix end (the same for every row): -inf in TMEM with
+        // whole-warp stores before the scores are read
+        if (__builtin_expect((kb + 1) * kTile > p_lkv, 0)) {
           const int valid = p_lkv - kb * kTile;
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            km[w] = valid >= 32 * (w + 1) ? ~0u
-                                          : (valid <= 32 * w ? 0u : ((1u << (valid - 32 * w)) - 1u));
+          const uint32_t ninf = __float_as_uint(-INFINITY);
+          const int v8 = (valid + 7) & ~7;
+          for (int col = valid; col < v8; ++col) tmem_st1(s_addr + col, ninf);
+          for (int col = v8; col < kTile; col += 8) tmem_st8_fill(s_addr + col, ninf);
+          tmem_wait_st();
         }
-        const bool masked = __any_sync(0xffffffffu, (km[0] & km[1] & km[2] & km[3]) != ~0u);
         // the block's 128 scores of this row, in registers for the whole block
         uint32_t sr[kTile];
         tmem_ld128_wait(s_addr, sr);
-        if (masked) {
-#pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            if (!((km[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
-        }
         auto row_max = [&]() {
           float mx0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[4]));
           float mx1 = fmaxf(__uint_as_float(sr[1]), __uint_as_float(sr[5]));
