@@ -369,6 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched behind the list builder with programmatic serialization: its lists and
+  // tile order are read only after it has completed
+  griddep_wait();
   const uint32_t tmem = tmem_base_sh;
   auto sQ = [&](int k) { return smem_base + L::kQ + (k & 1) * L::kTileBytes; };
   auto sSlot = [&](int s) { return smem_base + L::kRing + s * L::kTileBytes; };

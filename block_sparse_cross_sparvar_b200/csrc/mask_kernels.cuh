@@ -12,6 +12,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace sparvar {
 
 constexpr int kMaskThreads = 256;
@@ -189,6 +191,9 @@ __global__ void __launch_bounds__(kMaskThreads)
     csla_mask_kernel(const ScaleGeometry g, int q_scale, int n_sink, int r_prev, int r_own,
                      int block_q, int block_kv, int nkb, int32_t* kv_cnt, int32_t* kv_idx,
                      uint8_t* blk_mask, const TileOrderOut ord) {
+  // the attention launch behind it may start its prologue now; it reads the lists
+  // only after this grid has completed
+  griddep_launch_dependents();
   extern __shared__ uint32_t bits[];
   const int qb = blockIdx.x;
   const int nwords = (nkb + 31) >> 5;

@@ -194,6 +194,15 @@ __device__ __forceinline__ void tmem_wait_st() {
 // gives registers back to the CTA's pool, .inc takes them from it and waits until
 // the pool holds enough, so the budgets of all warpgroups must add up to at most
 // the registers the CTA was launched with.
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the kernel ahead of it on the stream has
+// finished, once every CTA of that kernel has signalled launch_dependents (or
+// exited); griddep_wait() then blocks until that kernel has completed and its
+// memory writes are visible.  Both are no-ops for kernels launched without it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));

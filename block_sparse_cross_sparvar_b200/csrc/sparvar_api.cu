@@ -164,7 +164,21 @@ int launch_fwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   if (ceil_div(tiles, grid) * (3 * row_len + 1) >= (int64_t{1} << 31))
     return fail(SPARVAR_ERR_UNSUPPORTED, "%lld query tiles x idx_row_len %lld too large per SM",
                 static_cast<long long>(tiles), static_cast<long long>(row_len));
-  kern<<<static_cast<unsigned>(grid), sparvar::fwd::kThreads, smem, stream>>>(tq, tk, tv, to, a);
+  // programmatic stream serialization: the CTAs may start (barriers, TMEM, tensor
+  // maps) while the kernel ahead of them on the stream (the list builder) finishes;
+  // the kernel waits for that kernel before it reads any list
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(sparvar::fwd::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, a);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return SPARVAR_OK;
