@@ -357,9 +357,10 @@ def test_ring_wait_before_p_is_caught():
 
 
 def test_longest_first_orders():
-    """The kernel can take its tiles longest list first (a serpentine over the CTAs);
-    a CTA then walks its lengths in falling order, with empty tiles last.  Such
-    sequences, and the same lengths rising, run clean."""
+    """The kernel can take its tiles in a given order (longest list first within
+    each wave, dealt in a serpentine over the CTAs), so a CTA's sequence of list
+    lengths can have any shape; the extreme ones, falling (with empty tiles last)
+    and rising, run clean, as do the random sequences of the other tests."""
     rng = random.Random(11)
     for t in range(40):
         tiles = [rng.choice([0, 0, 1, 2, 3, 4, 6, 9]) for _ in range(rng.randint(2, 8))]
