@@ -99,6 +99,8 @@ SPARVAR_API int sparvar_scale_blocks(const int32_t* sides, int n_scales, int q_s
  * kv_cnt     device, int32[nqb]          out: kept KV blocks per query block.
  * kv_idx     device, int32[nqb * nkb]    out: ascending kept indices, -1 padded.
  * blk_mask   device, uint8[nqb * nkb] or NULL; out: 1 = kept.
+ * The kernel lets a programmatically serialized launch behind it on the stream
+ * (the attention call) start at once; that launch waits for it before reading.
  */
 SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int q_scale,
                             int n_sink_scales, int radius_prev, int radius_own,
@@ -106,8 +108,9 @@ SPARVAR_API int sparvar_build_csla_mask(const int32_t* sides, int n_scales, int 
                             uint8_t* blk_mask, void* stream);
 
 /*
- * sparvar_build_csla_mask at block_q = block_kv = 128 (no blk_mask) that also
- * writes, in the same launch, the tile order of sparvar_tile_order
+ * sparvar_build_csla_mask at block_q = block_kv = 128 (no blk_mask), which lets
+ * the attention launch behind it start early (see sparvar_block_sparse_attn_fwd),
+ * that also writes, in the same launch, the tile order of sparvar_tile_order
  * for an attention call over B batch items and H heads sharing these lists
  * (order: device int32 [B * H * nqb]; for launches on the current device).  The
  * CTA that finishes last ranks the lists: done is a device int32 the caller sets
@@ -271,6 +274,10 @@ SPARVAR_API int sparvar_map_indices_2d(const int32_t* src_cnt, const int32_t* sr
  * dev_status device int32 or NULL: SPARVAR_DEV_BAD_LIST when an entry is out of
  *            range (the entry contributes nothing), SPARVAR_DEV_TIMEOUT when a
  *            bounded wait gave up.
+ * Stream order: the kernel is launched with programmatic stream serialization,
+ *   so its CTAs may start while the kernel ahead of it on `stream` finishes (when
+ *   that kernel allows it, as the list builders do); they read no input before
+ *   that kernel has completed, so the usual stream order holds for every buffer.
  */
 SPARVAR_API int sparvar_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
                                   float* lse, int B, int H, int Lq, int Lkv, int D,
