@@ -302,10 +302,14 @@ def test_csla_build_with_tile_order():
     lists are those of the plain builder, and the counter is back at zero, so the
     next call can use it again."""
     done = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for q_scale, B, H in ((9, 2, 16), (12, 2, 16), (12, 1, 5), (11, 3, 25)):
-        cnt0, idx0, _ = ops.sparvar_build_csla_mask(INF, q_scale, 5, 2, 4, 128, 128)
+    wide = (1, 2, 4, 8, 16, 32, 64, 128)  # 128 query blocks at the last scale: several
+    #                                       chunks of 32 in each round's walk
+    for sides, q_scale, csla, B, H in ((INF, 9, (5, 2, 4), 2, 16), (INF, 12, (5, 2, 4), 2, 16),
+                                       (INF, 12, (5, 2, 4), 1, 5), (INF, 11, (2, 1, 2), 3, 25),
+                                       (wide, 7, (2, 1, 2), 1, 3), (wide, 7, (3, 1, 3), 2, 5)):
+        cnt0, idx0, _ = ops.sparvar_build_csla_mask(sides, q_scale, *csla, 128, 128)
         for _ in range(2):
-            cnt, idx, order = ops.sparvar_build_csla_mask_ordered(INF, q_scale, 5, 2, 4, B, H,
+            cnt, idx, order = ops.sparvar_build_csla_mask_ordered(sides, q_scale, *csla, B, H,
                                                                   done=done)
             torch.cuda.synchronize()
             assert torch.equal(cnt, cnt0) and torch.equal(idx, idx0)
