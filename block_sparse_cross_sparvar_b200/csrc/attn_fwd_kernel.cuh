@@ -617,6 +617,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
          }
         }
+        // fine blocks of 32 or 64 rows: the rows of one warp share their keep bits, so
+        // the dropped fine KV blocks are set to -inf in TMEM as well (whole-warp stores)
+        // and the registers need no mask
+        if constexpr (FINE && kTmemMask) {
+          if (fine && args.mask_shift >= 5) {
+            const uint32_t ninf = __float_as_uint(-INFINITY);
+            const int w = 1 << args.mask_shift;
+            for (int i = 0; i < (kTile >> args.mask_shift); ++i)
+              if (!((keep >> i) & 1u))
+                for (int col = i * w; col < (i + 1) * w; col += 8) tmem_st8_fill(s_addr + col, ninf);
+            tmem_wait_st();
+            fine = false;
+          }
+        }
         auto dropped = [&](int col) {
           return col >= valid || !((keep >> (col >> args.mask_shift)) & 1u) ||
                  !((km[col >> 5] >> (col & 31)) & 1u);
