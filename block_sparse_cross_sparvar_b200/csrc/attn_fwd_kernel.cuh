@@ -605,9 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           fine = true;
         }
         // columns at or past the prefix end (the same for every row): -inf in TMEM
-        // before S is read, with whole-warp stores (the multi-problem and token-mask
-        // instantiations mask them in registers, which spills less there)
-        constexpr bool kTmemMask = !MULTI && !TOK;
+        // before S is read, with whole-warp stores (the token-mask instantiation masks
+        // its rows in registers anyway)
+        constexpr bool kTmemMask = !TOK;
         if constexpr (kTmemMask) {
          if (__builtin_expect(valid < kTile, 0)) {
           const uint32_t ninf = __float_as_uint(-INFINITY);
