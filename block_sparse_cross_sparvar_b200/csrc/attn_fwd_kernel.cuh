@@ -284,11 +284,14 @@ __device__ __forceinline__ void csla_row_mask(const CslaTokens& t, int i, int j,
     if (o1 <= k0 || o0 >= k1) continue;
     const int sm = t.side[m];
     const int r = m == t.q_scale ? t.r_own : t.r_prev;
-    const int ci = static_cast<int>(static_cast<int64_t>(i) * sm / sk);
-    const int cj = static_cast<int>(static_cast<int64_t>(j) * sm / sk);
+    // (32-bit unsigned arithmetic: sides are at most 46340, so i * sm < 2^32)
+    const uint32_t usm = static_cast<uint32_t>(sm), usk = static_cast<uint32_t>(sk);
+    const int ci = static_cast<int>(static_cast<uint32_t>(i) * usm / usk);
+    const int cj = static_cast<int>(static_cast<uint32_t>(j) * usm / usk);
     const int c0 = max(cj - r, 0), c1 = min(cj + r, sm - 1);
-    const int a0 = max(max(ci - r, 0), (max(k0, o0) - o0) / sm);
-    const int a1 = min(min(ci + r, sm - 1), (min(k1, o1) - 1 - o0) / sm);
+    const int a0 = max(max(ci - r, 0), static_cast<int>(static_cast<uint32_t>(max(k0, o0) - o0) / usm));
+    const int a1 = min(min(ci + r, sm - 1),
+                       static_cast<int>(static_cast<uint32_t>(min(k1, o1) - 1 - o0) / usm));
     for (int a = a0; a <= a1; ++a) {
       const int lo = max(o0 + a * sm + c0, k0) - k0;
       const int hi = min(o0 + a * sm + c1 + 1, k1) - k0;
