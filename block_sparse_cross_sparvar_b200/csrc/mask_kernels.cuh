@@ -220,9 +220,11 @@ __global__ void __launch_bounds__(kMaskThreads)
       const int j_hi = (i == i1) ? q1 - i * sk : sk - 1;
       const int sm = g.side[m];
       const int r = (m == q_scale) ? r_own : r_prev;
-      const int ci = static_cast<int>((static_cast<int64_t>(i) * sm) / sk);
-      const int cl = static_cast<int>((static_cast<int64_t>(j_lo) * sm) / sk);
-      const int ch = static_cast<int>((static_cast<int64_t>(j_hi) * sm) / sk);
+      // (32-bit unsigned: sides are at most 46340, so the products stay below 2^32)
+      const uint32_t usm = static_cast<uint32_t>(sm), usk = static_cast<uint32_t>(sk);
+      const int ci = static_cast<int>(static_cast<uint32_t>(i) * usm / usk);
+      const int cl = static_cast<int>(static_cast<uint32_t>(j_lo) * usm / usk);
+      const int ch = static_cast<int>(static_cast<uint32_t>(j_hi) * usm / usk);
       const int a_lo = max(0, ci - r), a_hi = min(sm - 1, ci + r);
       const int b_lo = max(0, cl - r), b_hi = min(sm - 1, ch + r);
       for (int a = a_lo; a <= a_hi; ++a) {
