@@ -228,3 +228,8 @@ def test_ordered_csla_build_rejects_bad_arguments(lib):
     assert call(done=0) == 1 and "order/done is NULL" in lib.sparvar_last_error().decode()
     assert call(B=0) == 1 and "B=0" in lib.sparvar_last_error().decode()
     assert call(q_scale=3) == 1 and "q_scale" in lib.sparvar_last_error().decode()
+    # the order is written by one CTA that ranks at most 1024 query blocks
+    wide = (ctypes.c_int32 * 2)(1, 400)  # 160000 queries: 1250 blocks of 128
+    rc = lib.sparvar_build_csla_mask_ordered(wide, 2, 1, 1, 1, 1, 1, 1, vp(16), vp(16), vp(16),
+                                             vp(16), vp(0))
+    assert rc == 2 and "1024 query blocks" in lib.sparvar_last_error().decode()
