@@ -471,7 +471,9 @@ def main():
                                 "compute and copy out on three streams",
                     "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                     "d2h_bytes_per_step": int(ho.numel() * 2)},
-            "gpu_launches": 2 * args.steps,
+            # the library's kernels in the timed regions: K steps (list build + attention),
+            # then K attention launches and K list builds timed alone
+            "gpu_launches": 4 * args.steps,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
