@@ -826,11 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // row `row`, columns [g D/2, (g+1) D/2), into the 128B-swizzled layout of the
           // output tensor map: 64-column chunks of 128 rows x 128 bytes, 16-byte unit u of
           // row r at position u ^ (r mod 8)
-#pragma unroll
-          for (int cc = 0; cc < D / 64; ++cc) {
-            const int col = g * (D / 2) + cc * 32;
-            uint32_t ro[32];
-            tmem_ld32_wait(o_addr + col, ro);
+          auto stage = [&](const uint32_t* ro, int col) {  // 32 columns from `col`
             uint32_t pk[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k)
@@ -844,6 +840,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                     ((unit ^ (row & 7)) << 4));
               *dst = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
+          };
+          // this thread's D/2 columns of O in one TMEM load
+          if constexpr (D == 128) {
+            uint32_t ro[64];
+            tmem_ld64_wait(o_addr + g * 64, ro);
+            stage(ro, g * 64);
+            stage(ro + 32, g * 64 + 32);
+          } else {
+            uint32_t ro[32];
+            tmem_ld32_wait(o_addr + g * 32, ro);
+            stage(ro, g * 32);
           }
         }
         fence_proxy_async_smem();
