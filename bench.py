@@ -492,7 +492,7 @@ def main():
             torch.cuda.empty_cache()
             for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass, workloads.cs4a_fused_pass,
                        workloads.decision_fused_vs_separate, workloads.csla_radius_sweep,
-                       workloads.csla_granularity_sweep, workloads.density_sweep):
+                       workloads.csla_granularity_sweep, workloads.density_sweep, workloads.ocache_scales):
                 print(json.dumps({"extra": fn(dev)}), flush=True)
                 torch.cuda.empty_cache()
     if world > 1:

@@ -1,7 +1,11 @@
 // CS4A output cache: a later scale's block-sparse output corrected by the
 // decision scale's residual (dense output minus sparse output), upsampled to
-// the later scale's grid by nearest neighbour.  Elementwise and bound by HBM:
-// each thread takes 8 channels (16 bytes) of one target token.
+// the later scale's grid by nearest neighbour.  Elementwise and bound by HBM.
+// One CTA per target row i of one (batch, head), whose nearest source row is
+// fixed; thread x takes 8 channels (16 bytes), thread y every ty-th token of
+// the row, four of them per pass.  The nearest source column of token j,
+// floor(j * s_src / s_dst), is carried from token to token as a quotient and
+// remainder, so the loop holds no integer division.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -27,36 +31,59 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
+// grid (s_dst, H, B), block (D / 8, ty) with ty * D / 8 <= 256
 __global__ void __launch_bounds__(256) ocache_apply_kernel(const OcacheArgs a) {
-  const int vecs = a.D / 8;
-  const int64_t n_t = static_cast<int64_t>(a.s_dst) * a.s_dst;
-  const int64_t total = static_cast<int64_t>(a.B) * a.H * n_t * vecs;
-  for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; x < total;
-       x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c8 = static_cast<int>(x % vecs);
-    const int64_t tok = (x / vecs) % n_t;
-    const int64_t bh = x / (vecs * n_t);
-    const int h = static_cast<int>(bh % a.H), b = static_cast<int>(bh / a.H);
-    const int i = static_cast<int>(tok / a.s_dst), j = static_cast<int>(tok % a.s_dst);
-    // nearest source token: row floor(i * s_src / s_dst), column likewise
-    const int64_t src = static_cast<int64_t>(i) * a.s_src / a.s_dst * a.s_src +
-                        static_cast<int64_t>(j) * a.s_src / a.s_dst;
-    const uint4 vt = *reinterpret_cast<const uint4*>(a.o_t + b * a.t_sb + h * a.t_sh + tok * a.t_sr + c8 * 8);
-    const uint4 vd = __ldg(reinterpret_cast<const uint4*>(a.o_d + b * a.d_sb + h * a.d_sh + src * a.d_sr + c8 * 8));
-    const uint4 vs = __ldg(reinterpret_cast<const uint4*>(a.o_s + b * a.s_sb + h * a.s_sh + src * a.s_sr + c8 * 8));
-    float ft[8], fd[8], fs[8];
-    bf16x8_to_f32(vt, ft);
-    bf16x8_to_f32(vd, fd);
-    bf16x8_to_f32(vs, fs);
-    uint32_t w[4];
+  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int c = threadIdx.x * 8;
+  const int ty = blockDim.y;
+  const int si = static_cast<int>(static_cast<int64_t>(i) * a.s_src / a.s_dst);
+  const int64_t row_t = static_cast<int64_t>(i) * a.s_dst, row_s = static_cast<int64_t>(si) * a.s_src;
+  const __nv_bfloat16* pt = a.o_t + b * a.t_sb + h * a.t_sh + row_t * a.t_sr + c;
+  __nv_bfloat16* pu = a.out + b * a.u_sb + h * a.u_sh + row_t * a.u_sr + c;
+  const __nv_bfloat16* pd = a.o_d + b * a.d_sb + h * a.d_sh + row_s * a.d_sr + c;
+  const __nv_bfloat16* ps = a.o_s + b * a.s_sb + h * a.s_sh + row_s * a.s_sr + c;
+  // j * s_src == sj * s_dst + rem, 0 <= rem < s_dst (j * s_src < 2^31 for sides <= 46340)
+  int j = threadIdx.y;
+  int sj = j * a.s_src / a.s_dst;
+  int rem = j * a.s_src - sj * a.s_dst;
+  const int step_q = ty * a.s_src / a.s_dst, step_r = ty * a.s_src - step_q * a.s_dst;
+  // four tokens per pass: every load of the pass is issued before its first store
+  constexpr int kU = 4;
+  for (; j < a.s_dst; j += kU * ty) {
+    uint4 vt[kU], vd[kU], vs[kU];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const __nv_bfloat162 p = __floats2bfloat162_rn(ft[2 * k] + (fd[2 * k] - fs[2 * k]),
-                                                     ft[2 * k + 1] + (fd[2 * k + 1] - fs[2 * k + 1]));
-      w[k] = *reinterpret_cast<const uint32_t*>(&p);
+    for (int u = 0; u < kU; ++u) {
+      const int ju = j + u * ty;
+      if (ju < a.s_dst) {
+        vt[u] = *reinterpret_cast<const uint4*>(pt + ju * a.t_sr);
+        vd[u] = __ldg(reinterpret_cast<const uint4*>(pd + sj * a.d_sr));
+        vs[u] = __ldg(reinterpret_cast<const uint4*>(ps + sj * a.s_sr));
+      }
+      sj += step_q;
+      rem += step_r;
+      if (rem >= a.s_dst) {
+        rem -= a.s_dst;
+        ++sj;
+      }
     }
-    *reinterpret_cast<uint4*>(a.out + b * a.u_sb + h * a.u_sh + tok * a.u_sr + c8 * 8) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int ju = j + u * ty;
+      if (ju < a.s_dst) {
+        float ft[8], fd[8], fs[8];
+        bf16x8_to_f32(vt[u], ft);
+        bf16x8_to_f32(vd[u], fd);
+        bf16x8_to_f32(vs[u], fs);
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __nv_bfloat162 p = __floats2bfloat162_rn(
+              ft[2 * k] + (fd[2 * k] - fs[2 * k]), ft[2 * k + 1] + (fd[2 * k + 1] - fs[2 * k + 1]));
+          w[k] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+        *reinterpret_cast<uint4*>(pu + ju * a.u_sr) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
   }
 }
 

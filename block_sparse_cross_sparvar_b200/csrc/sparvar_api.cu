@@ -919,15 +919,13 @@ int sparvar_ocache_apply(const void* o_target, const void* o_dense, const void* 
   a.d_sb = d_strides[0]; a.d_sh = d_strides[1]; a.d_sr = d_strides[2];
   a.s_sb = s_strides[0]; a.s_sh = s_strides[1]; a.s_sr = s_strides[2];
   a.u_sb = out_strides[0]; a.u_sh = out_strides[1]; a.u_sr = out_strides[2];
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "multiprocessor count");
-  const int64_t total = static_cast<int64_t>(B) * H * n_dst * (D / 8);
-  const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), static_cast<int64_t>(sms) * 8);
-  sparvar::ocache_apply_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+  // one CTA per target row of one (batch, head): D / 8 threads across the channels,
+  // up to 256 / (D / 8) tokens of the row at a time
+  const int vecs = D / 8;
+  const int ty = std::max(1, std::min(256 / vecs, side_dst));
+  sparvar::ocache_apply_kernel<<<dim3(side_dst, H, B), dim3(vecs, ty), 0,
                                  static_cast<cudaStream_t>(stream)>>>(a);
-  e = cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "ocache_apply_kernel launch");
   return SPARVAR_OK;
 }

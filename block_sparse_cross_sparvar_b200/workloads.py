@@ -14,6 +14,8 @@
   (sink block always kept), with the full key prefix and with the 40x40 and
   48x48 scales skipped from the prefix; each also with the query tiles taken
   longest list first.
+* ``ocache_scales``: the CS4A output cache alone, from the 32x32 decision scale
+  to the 40x40, 48x48 and 64x64 scales, against the HBM bytes it must move.
 
 Every step runs in the library's kernels; torch only provides memory, streams
 and events.
@@ -54,7 +56,11 @@ def kept_flops(cnt, idx, nq, L, block, D):
     return total, int(np.prod(lead)) if lead else 1
 
 
-def time_ms(fn, reps, device, warmup=3):
+def time_ms(fn, reps, device, warmup=3, sleep_ahead=False):
+    """Median device time of fn over reps runs, a 256 MB L2 flush before each.
+    sleep_ahead: a GPU sleep is queued after the flush, so that the host has
+    queued the start event, fn's launches and the end event before the GPU
+    reaches them (for calls shorter than their own host-side launch cost)."""
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=device)
     for _ in range(warmup):
         fn()
@@ -62,6 +68,8 @@ def time_ms(fn, reps, device, warmup=3):
     out = []
     for i in range(reps):
         flush.fill_(i)
+        if sleep_ahead:
+            torch.cuda._sleep(400_000)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
@@ -340,3 +348,23 @@ def density_sweep(device, reps=10, seed=0, B=2, H=16, D=128, densities=(0.05, 0.
                         "tflops": f / (ms * 1e-3) / 1e12, "ms_longest_first": ms_lpt,
                         "tflops_longest_first": f / (ms_lpt * 1e-3) / 1e12})
     return {"workload": "last_scale_density_sweep", "B": B, "H": H, "D": D, "runs": res}
+
+
+def ocache_scales(device, reps=20, seed=0, B=2, H=16, D=128, s_src=32, targets=(40, 48, 64)):
+    """The output cache alone (out of place), L2 flushed between runs, timed
+    behind a GPU sleep (the call is shorter than its host-side cost).  Its bytes:
+    the target output read and the corrected output written once, the decision
+    scale's dense and sparse outputs read once (their re-reads by neighbouring
+    target tokens come from L2)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    rnd = lambda n: torch.randn(B, H, n, D, generator=g, device=device).to(torch.bfloat16)  # noqa: E731
+    o_d, o_s = rnd(s_src * s_src), rnd(s_src * s_src)
+    res = []
+    for t in targets:
+        o_t = rnd(t * t)
+        out = torch.empty_like(o_t)
+        ms = time_ms(lambda: ops.sparvar_ocache_apply(o_t, o_d, o_s, s_src, t, out=out), reps, device,
+                     sleep_ahead=True)
+        nbytes = 2 * B * H * D * (2 * t * t + 2 * s_src * s_src)
+        res.append({"s_src": s_src, "s_dst": t, "ms": ms, "bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9})
+    return {"workload": "cs4a_output_cache", "B": B, "H": H, "D": D, "runs": res}

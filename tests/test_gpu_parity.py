@@ -682,7 +682,8 @@ def test_cs4a_topk_2d_pipeline_attention():
 
 # ------------------------------------------------------------------ CS4A output cache
 @pytest.mark.parametrize("s_src,s_dst,D", [(32, 64, 128), (32, 40, 128), (32, 48, 64), (7, 7, 128),
-                                           (5, 13, 64)])
+                                           (5, 13, 64), (3, 17, 8), (6, 9, 72), (4, 7, 1024),
+                                           (13, 5, 128)])
 def test_ocache_apply_elementwise(s_src, s_dst, D):
     rng = np.random.default_rng(s_src * s_dst + D)
     B, H = 2, 3
