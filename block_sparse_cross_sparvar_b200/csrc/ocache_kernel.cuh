@@ -11,6 +11,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace sparvar {
 
 struct OcacheArgs {
@@ -22,13 +24,9 @@ struct OcacheArgs {
   int64_t t_sb, t_sh, t_sr, d_sb, d_sh, d_sr, s_sb, s_sh, s_sr, u_sb, u_sh, u_sr;
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+// two bf16 (low half first) as an f32 pair
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // grid (s_dst, H, B), block (D / 8, ty) with ty * D / 8 <= 256
@@ -38,51 +36,59 @@ __global__ void __launch_bounds__(256) ocache_apply_kernel(const OcacheArgs a) {
   const int ty = blockDim.y;
   const int si = static_cast<int>(static_cast<int64_t>(i) * a.s_src / a.s_dst);
   const int64_t row_t = static_cast<int64_t>(i) * a.s_dst, row_s = static_cast<int64_t>(si) * a.s_src;
-  const __nv_bfloat16* pt = a.o_t + b * a.t_sb + h * a.t_sh + row_t * a.t_sr + c;
-  __nv_bfloat16* pu = a.out + b * a.u_sb + h * a.u_sh + row_t * a.u_sr + c;
-  const __nv_bfloat16* pd = a.o_d + b * a.d_sb + h * a.d_sh + row_s * a.d_sr + c;
-  const __nv_bfloat16* ps = a.o_s + b * a.s_sb + h * a.s_sh + row_s * a.s_sr + c;
   // j * s_src == sj * s_dst + rem, 0 <= rem < s_dst (j * s_src < 2^31 for sides <= 46340)
   int j = threadIdx.y;
-  int sj = j * a.s_src / a.s_dst;
+  const int sj = j * a.s_src / a.s_dst;
   int rem = j * a.s_src - sj * a.s_dst;
   const int step_q = ty * a.s_src / a.s_dst, step_r = ty * a.s_src - step_q * a.s_dst;
+  // running pointers at token j and its source column sj; a step of ty tokens
+  // moves the source column by step_q, or step_q + 1 when the remainder wraps
+  const __nv_bfloat16* pt = a.o_t + b * a.t_sb + h * a.t_sh + (row_t + j) * a.t_sr + c;
+  __nv_bfloat16* pu = a.out + b * a.u_sb + h * a.u_sh + (row_t + j) * a.u_sr + c;
+  const __nv_bfloat16* pd = a.o_d + b * a.d_sb + h * a.d_sh + (row_s + sj) * a.d_sr + c;
+  const __nv_bfloat16* ps = a.o_s + b * a.s_sb + h * a.s_sh + (row_s + sj) * a.s_sr + c;
+  const int64_t t_step = ty * a.t_sr, u_step = ty * a.u_sr;
+  const int64_t d_step = step_q * a.d_sr, s_step = step_q * a.s_sr;
+  const uint64_t neg1 = f2_pack(-1.f, -1.f);
   // four tokens per pass: every load of the pass is issued before its first store
   constexpr int kU = 4;
   for (; j < a.s_dst; j += kU * ty) {
     uint4 vt[kU], vd[kU], vs[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int ju = j + u * ty;
-      if (ju < a.s_dst) {
-        vt[u] = *reinterpret_cast<const uint4*>(pt + ju * a.t_sr);
-        vd[u] = __ldg(reinterpret_cast<const uint4*>(pd + sj * a.d_sr));
-        vs[u] = __ldg(reinterpret_cast<const uint4*>(ps + sj * a.s_sr));
+      if (j + u * ty < a.s_dst) {
+        vt[u] = *reinterpret_cast<const uint4*>(pt);
+        vd[u] = __ldg(reinterpret_cast<const uint4*>(pd));
+        vs[u] = __ldg(reinterpret_cast<const uint4*>(ps));
       }
-      sj += step_q;
+      pt += t_step;
+      pd += d_step;
+      ps += s_step;
       rem += step_r;
       if (rem >= a.s_dst) {
         rem -= a.s_dst;
-        ++sj;
+        pd += a.d_sr;
+        ps += a.s_sr;
       }
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int ju = j + u * ty;
-      if (ju < a.s_dst) {
-        float ft[8], fd[8], fs[8];
-        bf16x8_to_f32(vt[u], ft);
-        bf16x8_to_f32(vd[u], fd);
-        bf16x8_to_f32(vs[u], fs);
+      if (j + u * ty < a.s_dst) {
+        const uint32_t wt[4] = {vt[u].x, vt[u].y, vt[u].z, vt[u].w};
+        const uint32_t wd[4] = {vd[u].x, vd[u].y, vd[u].z, vd[u].w};
+        const uint32_t ws[4] = {vs[u].x, vs[u].y, vs[u].z, vs[u].w};
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const __nv_bfloat162 p = __floats2bfloat162_rn(
-              ft[2 * k] + (fd[2 * k] - fs[2 * k]), ft[2 * k + 1] + (fd[2 * k + 1] - fs[2 * k + 1]));
-          w[k] = *reinterpret_cast<const uint32_t*>(&p);
+          // (lo, hi) channel pairs in f32: t + (d - s), each step rounded once
+          const uint64_t r = f2_fma(bf16x2_to_f2(ws[k]), neg1, bf16x2_to_f2(wd[k]));
+          float lo, hi;
+          f2_unpack(f2_add(bf16x2_to_f2(wt[k]), r), lo, hi);
+          w[k] = pack_bf16x2(lo, hi);
         }
-        *reinterpret_cast<uint4*>(pu + ju * a.u_sr) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(pu) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      pu += u_step;
     }
   }
 }
