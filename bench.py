@@ -127,7 +127,7 @@ def start_clock_sampler(path):
         return None, None
 
 
-def stop_clock_sampler(proc, f, path, gpu_index):
+def stop_clock_sampler(proc, f, path, gpu_index, window="1 s of back-to-back steps + the timed region"):
     if proc is None:
         return None
     proc.terminate()
@@ -153,7 +153,7 @@ def stop_clock_sampler(proc, f, path, gpu_index):
     if not sm:
         return None
     return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "samples": len(sm),
-            "reasons": sorted(reasons), "window": "1 s of back-to-back steps + the timed region"}
+            "reasons": sorted(reasons), "window": window}
 
 
 def cpu_baseline(wl, budget_s=12.0, seed=0, d=None):
@@ -493,7 +493,12 @@ def main():
             for fn in (workloads.cs4a_full_pass, workloads.cs4a_topk_2d_pass, workloads.cs4a_fused_pass,
                        workloads.decision_fused_vs_separate, workloads.csla_radius_sweep,
                        workloads.csla_granularity_sweep, workloads.density_sweep, workloads.ocache_scales):
-                print(json.dumps({"extra": fn(dev)}), flush=True)
+                # SM clocks and throttle reasons over the whole run of the workload
+                xs, xf = start_clock_sampler(clocks_path)
+                rec = fn(dev)
+                rec["clocks"] = stop_clock_sampler(xs, xf, clocks_path, torch.cuda.current_device(),
+                                                   window="the whole workload, warm-up included")
+                print(json.dumps({"extra": rec}), flush=True)
                 torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
